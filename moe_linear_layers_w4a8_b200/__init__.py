@@ -1,0 +1,323 @@
+"""W4A8 quantized Linear / MoE-expert GEMM for NVIDIA B200 (sm_100a).
+
+Thin Python binding of the C ABI in include/w4a8.h (libw4a8.so, built
+in-tree).  This module only marshals arguments: torch supplies device memory
+and the current CUDA stream; every step of the computation runs in the
+library's CUDA kernels.  There is no fallback: if the library cannot be
+loaded, every call raises W4A8Error.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+import threading
+from typing import Optional
+
+import torch
+
+__all__ = [
+    "W4A8Error", "WDesc", "PackedWeight", "load_library", "library_path",
+    "w4a8_pack_weights", "w4a8_pack_expert_weights", "w4a8_quant_act", "w4a8_gemm",
+    "w4a8_gemm_debug_partials", "w4a8_moe_grouped_gemm", "w4a8_moe_workspace_layout",
+    "w4a8_gemm_workspace_size", "w4a8_moe_workspace_size", "w4a8_get_device_status",
+    "w4a8_status_string", "w4a8_selftest_bounded_wait", "w4a8_linear", "LAYOUT_VERSION",
+    "STATUS",
+]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LAYOUT_VERSION = 1
+STATUS = {
+    0: "W4A8_OK", 1: "W4A8_ERR_INVALID_ARG", 2: "W4A8_ERR_UNSUPPORTED_SHAPE",
+    3: "W4A8_ERR_FORMAT_MISMATCH", 4: "W4A8_ERR_NONFINITE", 5: "W4A8_ERR_TIMEOUT",
+    6: "W4A8_ERR_CUDA", 7: "W4A8_ERR_WORKSPACE",
+}
+
+
+class W4A8Error(RuntimeError):
+    def __init__(self, code: int, where: str = ""):
+        self.code = int(code)
+        super().__init__(f"{where}: {STATUS.get(self.code, 'W4A8_ERR_UNKNOWN')} ({self.code})")
+
+
+class WDesc(ctypes.Structure):
+    _fields_ = [("bits", ctypes.c_int32), ("symmetric", ctypes.c_int32), ("group", ctypes.c_int32),
+                ("K", ctypes.c_int32), ("N", ctypes.c_int32), ("layout_version", ctypes.c_int32)]
+
+    def copy(self) -> "WDesc":
+        return WDesc(self.bits, self.symmetric, self.group, self.K, self.N, self.layout_version)
+
+
+class MoeWsLayout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in ("perm", "inv", "qx", "sx", "h", "qh", "sh", "yd", "total")]
+
+
+@dataclasses.dataclass
+class PackedWeight:
+    """Packed 4-bit weight (one matrix, or E stacked expert matrices)."""
+    packed: torch.Tensor           # uint8 [(E,) N*K/2]
+    s_w: torch.Tensor              # fp32 [(E,) G, N]
+    z: Optional[torch.Tensor]      # uint8 [(E,) G, N] or None (symmetric)
+    desc: WDesc
+    experts: int = 0               # 0 = single matrix
+
+    @property
+    def K(self):
+        return self.desc.K
+
+    @property
+    def N(self):
+        return self.desc.N
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def library_path() -> str:
+    return os.path.join(_PKG, "libw4a8.so")
+
+
+def load_library():
+    """Loads libw4a8.so (raises W4A8Error(6) when it is missing)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        path = library_path()
+        if not os.path.exists(path):
+            raise W4A8Error(6, f"libw4a8.so not built (expected at {path}); run the package build")
+        L = ctypes.CDLL(path)
+        P, I, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        st = ctypes.c_int
+        L.w4a8_abi_version.restype = I
+        L.w4a8_status_string.restype = ctypes.c_char_p
+        L.w4a8_status_string.argtypes = [st]
+        L.w4a8_packed_bytes.restype = S
+        L.w4a8_packed_bytes.argtypes = [I, I]
+        L.w4a8_gemm_workspace_size.restype = S
+        L.w4a8_gemm_workspace_size.argtypes = [I, ctypes.POINTER(WDesc)]
+        L.w4a8_moe_workspace_size.restype = S
+        L.w4a8_moe_workspace_size.argtypes = [I, I, I, ctypes.POINTER(WDesc), ctypes.POINTER(WDesc)]
+        L.w4a8_moe_workspace_layout.restype = st
+        L.w4a8_moe_workspace_layout.argtypes = [I, I, I, ctypes.POINTER(WDesc), ctypes.POINTER(WDesc),
+                                                ctypes.POINTER(MoeWsLayout)]
+        L.w4a8_pack_weights.restype = st
+        L.w4a8_pack_weights.argtypes = [P, I, I, I, I, P, P, P, ctypes.POINTER(WDesc), P, P]
+        L.w4a8_quant_act.restype = st
+        L.w4a8_quant_act.argtypes = [P, I, I, I, I, P, P, P, P, P]
+        L.w4a8_gemm.restype = st
+        L.w4a8_gemm.argtypes = [P, P, P, P, P, ctypes.POINTER(WDesc), I, P, I, P, S, P, P]
+        L.w4a8_gemm_debug_partials.restype = st
+        L.w4a8_gemm_debug_partials.argtypes = [P, P, P, P, P, ctypes.POINTER(WDesc), I, P, I, P, P, S, P, P]
+        L.w4a8_moe_grouped_gemm.restype = st
+        L.w4a8_moe_grouped_gemm.argtypes = [P, P, I, I, I, P, P, P, ctypes.POINTER(WDesc), P, P, P,
+                                            ctypes.POINTER(WDesc), P, P, P, P, P, S, P, P]
+        L.w4a8_get_device_status.restype = st
+        L.w4a8_get_device_status.argtypes = [P, P]
+        L.w4a8_selftest_bounded_wait.restype = st
+        L.w4a8_selftest_bounded_wait.argtypes = [P, ctypes.c_uint64, P]
+        _lib = L
+        return L
+
+
+def _p(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(dev: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+
+
+def _check(code: int, where: str):
+    if code != 0:
+        raise W4A8Error(code, where)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise W4A8Error(1, "tensors must be on a CUDA device")
+
+
+def w4a8_status_string(code: int) -> str:
+    return load_library().w4a8_status_string(int(code)).decode()
+
+
+def w4a8_get_device_status(status: torch.Tensor) -> int:
+    """Synchronizes the current stream and returns the device status word."""
+    return int(load_library().w4a8_get_device_status(_p(status), _stream(status.device)))
+
+
+def new_status(device) -> torch.Tensor:
+    return torch.zeros(1, dtype=torch.int32, device=device)
+
+
+# ----------------------------------------------------------------- packing --
+
+def w4a8_pack_weights(W: torch.Tensor, group: int = 128, symmetric: bool = True,
+                      status: Optional[torch.Tensor] = None, out: Optional[PackedWeight] = None,
+                      expert: Optional[int] = None) -> PackedWeight:
+    """Group-wise 4-bit quantization + packing of W fp32 [K, N] (device).
+    With `out` and `expert`, writes expert slot `expert` of a stacked weight."""
+    L = load_library()
+    _need_cuda(W)
+    if W.dtype != torch.float32 or W.dim() != 2:
+        raise W4A8Error(1, "W must be fp32 [K, N]")
+    W = W.contiguous()
+    K, N = W.shape
+    G = K // group if group > 0 else 0
+    if out is None:
+        packed = torch.empty(K * N // 2, dtype=torch.uint8, device=W.device)
+        s_w = torch.empty(G, N, dtype=torch.float32, device=W.device)
+        z = None if symmetric else torch.empty(G, N, dtype=torch.uint8, device=W.device)
+        pk, sw, zz = packed, s_w, z
+    else:
+        e = int(expert)
+        pk, sw = out.packed[e], out.s_w[e]
+        zz = None if out.z is None else out.z[e]
+    d = WDesc()
+    code = L.w4a8_pack_weights(_p(W), K, N, group, int(bool(symmetric)), _p(pk), _p(sw), _p(zz),
+                               ctypes.byref(d), _p(status), _stream(W.device))
+    _check(code, "w4a8_pack_weights")
+    if out is not None:
+        return out
+    return PackedWeight(packed=pk, s_w=sw, z=zz, desc=d)
+
+
+def w4a8_pack_expert_weights(make_weight, E: int, K: int, N: int, group: int, symmetric: bool,
+                             device, status: Optional[torch.Tensor] = None) -> PackedWeight:
+    """Packs E expert matrices (make_weight(e) -> fp32 [K, N] on `device`)
+    into one stacked PackedWeight."""
+    G = K // group
+    packed = torch.empty(E, K * N // 2, dtype=torch.uint8, device=device)
+    s_w = torch.empty(E, G, N, dtype=torch.float32, device=device)
+    z = None if symmetric else torch.empty(E, G, N, dtype=torch.uint8, device=device)
+    pw = PackedWeight(packed=packed, s_w=s_w, z=z,
+                      desc=WDesc(4, int(bool(symmetric)), group, K, N, LAYOUT_VERSION), experts=E)
+    for e in range(E):
+        w4a8_pack_weights(make_weight(e), group, symmetric, status=status, out=pw, expert=e)
+    return pw
+
+
+# ------------------------------------------------------------- activation --
+
+def w4a8_quant_act(X: torch.Tensor, group_for_rowsum: int = 0, status: Optional[torch.Tensor] = None):
+    """Per-token INT8 quantization of X bf16 [M, K] -> (q int8, s_x fp32, rowsum|None)."""
+    L = load_library()
+    _need_cuda(X)
+    if X.dtype != torch.bfloat16 or X.dim() != 2 or X.stride(1) != 1:
+        raise W4A8Error(1, "X must be bf16 [M, K] with unit column stride")
+    M, K = X.shape
+    q = torch.empty(M, K, dtype=torch.int8, device=X.device)
+    s = torch.empty(M, dtype=torch.float32, device=X.device)
+    rs = (torch.empty(M, K // group_for_rowsum, dtype=torch.int32, device=X.device)
+          if group_for_rowsum else None)
+    code = L.w4a8_quant_act(_p(X), M, K, X.stride(0), int(group_for_rowsum), _p(q), _p(s), _p(rs),
+                            _p(status), _stream(X.device))
+    _check(code, "w4a8_quant_act")
+    return q, s, rs
+
+
+# ------------------------------------------------------------------- GEMM ---
+
+def w4a8_gemm_workspace_size(M: int, w: PackedWeight) -> int:
+    return int(load_library().w4a8_gemm_workspace_size(int(M), ctypes.byref(w.desc)))
+
+
+def _gemm(qx, s_x, w: PackedWeight, out, workspace, status, P):
+    L = load_library()
+    _need_cuda(qx, s_x)
+    if qx.dtype != torch.int8 or qx.dim() != 2 or not qx.is_contiguous():
+        raise W4A8Error(1, "qx must be contiguous int8 [M, K]")
+    M = qx.shape[0]
+    if out is None:
+        out = torch.empty(M, w.N, dtype=torch.bfloat16, device=qx.device)
+    need = w4a8_gemm_workspace_size(M, w)
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=qx.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    if P is None:
+        code = L.w4a8_gemm(_p(qx), _p(s_x), _p(w.packed), _p(w.s_w), _p(w.z), ctypes.byref(w.desc), M,
+                           _p(out), out.stride(0), _p(workspace), ws_bytes, _p(status), _stream(qx.device))
+        _check(code, "w4a8_gemm")
+    else:
+        code = L.w4a8_gemm_debug_partials(_p(qx), _p(s_x), _p(w.packed), _p(w.s_w), _p(w.z),
+                                          ctypes.byref(w.desc), M, _p(out), out.stride(0), _p(P),
+                                          _p(workspace), ws_bytes, _p(status), _stream(qx.device))
+        _check(code, "w4a8_gemm_debug_partials")
+    return out
+
+
+def w4a8_gemm(qx: torch.Tensor, s_x: torch.Tensor, w: PackedWeight, out: Optional[torch.Tensor] = None,
+              workspace: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Y bf16 [M, N] = W4A8(qx, w)."""
+    return _gemm(qx, s_x, w, out, workspace, status, None)
+
+
+def w4a8_gemm_debug_partials(qx, s_x, w: PackedWeight, out=None, workspace=None, status=None):
+    """(Y, P int32 [M, G, N]) — the exact group partials as the tensor cores produced them."""
+    M = qx.shape[0]
+    P = torch.zeros(M, w.K // w.desc.group, w.N, dtype=torch.int32, device=qx.device)
+    Y = _gemm(qx, s_x, w, out, workspace, status, P)
+    return Y, P
+
+
+def w4a8_linear(X: torch.Tensor, w: PackedWeight, out=None, workspace=None, status=None) -> torch.Tensor:
+    """Per-token quantization of X followed by the W4A8 GEMM."""
+    q, s, _ = w4a8_quant_act(X, status=status)
+    return w4a8_gemm(q, s, w, out=out, workspace=workspace, status=status)
+
+
+# -------------------------------------------------------------------- MoE ---
+
+def w4a8_moe_workspace_size(T: int, E: int, topk: int, w1: PackedWeight, w2: PackedWeight) -> int:
+    return int(load_library().w4a8_moe_workspace_size(T, E, topk, ctypes.byref(w1.desc),
+                                                      ctypes.byref(w2.desc)))
+
+
+def w4a8_moe_workspace_layout(T: int, E: int, topk: int, w1: PackedWeight, w2: PackedWeight) -> dict:
+    lay = MoeWsLayout()
+    code = load_library().w4a8_moe_workspace_layout(T, E, topk, ctypes.byref(w1.desc), ctypes.byref(w2.desc),
+                                                    ctypes.byref(lay))
+    _check(code, "w4a8_moe_workspace_layout")
+    return {n: int(getattr(lay, n)) for n, _ in MoeWsLayout._fields_}
+
+
+def w4a8_moe_grouped_gemm(X: torch.Tensor, logits: torch.Tensor, topk: int, w1: PackedWeight,
+                          w2: PackedWeight, workspace: Optional[torch.Tensor] = None,
+                          status: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None):
+    """One MoE expert layer (route, dispatch, gate_up + SiLU*up, down, combine).
+    Returns dict(out, topk_idx, topk_w, expert_offsets, workspace)."""
+    L = load_library()
+    _need_cuda(X, logits)
+    if X.dtype != torch.bfloat16 or logits.dtype != torch.float32:
+        raise W4A8Error(1, "X must be bf16 and logits fp32")
+    X = X.contiguous()
+    logits = logits.contiguous()
+    T, H = X.shape
+    E = logits.shape[1]
+    dev = X.device
+    need = w4a8_moe_workspace_size(T, E, topk, w1, w2)
+    if need == 0 and T > 0:
+        raise W4A8Error(2, "w4a8_moe_workspace_size: shape not supported")
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    if out is None:
+        out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+    idx = torch.empty(T, topk, dtype=torch.int32, device=dev)
+    pw = torch.empty(T, topk, dtype=torch.float32, device=dev)
+    offs = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    code = L.w4a8_moe_grouped_gemm(
+        _p(X), _p(logits), T, E, int(topk),
+        _p(w1.packed), _p(w1.s_w), _p(w1.z), ctypes.byref(w1.desc),
+        _p(w2.packed), _p(w2.s_w), _p(w2.z), ctypes.byref(w2.desc),
+        _p(out), _p(idx), _p(pw), _p(offs), _p(workspace),
+        workspace.numel() * workspace.element_size(), _p(status), _stream(dev))
+    _check(code, "w4a8_moe_grouped_gemm")
+    return dict(out=out, topk_idx=idx, topk_w=pw, expert_offsets=offs, workspace=workspace)
+
+
+def w4a8_selftest_bounded_wait(status: torch.Tensor, limit_ns: int = 1_000_000) -> None:
+    code = load_library().w4a8_selftest_bounded_wait(_p(status), int(limit_ns), _stream(status.device))
+    _check(code, "w4a8_selftest_bounded_wait")

@@ -1,0 +1,413 @@
+// Memory-bound kernels around the W4A8 GEMM: per-token INT8 quantization,
+// offline 4-bit group packing, MoE routing / dispatch / combine, and the
+// fixed-order split-K reduction.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "ptx.cuh"
+
+namespace w4a8 {
+
+constexpr int kStatusNonfinite = 4;
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t h16) { return __uint_as_float(h16 << 16); }
+
+__device__ __forceinline__ uint16_t f32_to_bf16_bits(float f) {
+    __nv_bfloat16 b = __float2bfloat16_rn(f);
+    return *reinterpret_cast<uint16_t*>(&b);
+}
+
+// ---------------------------------------------------------------------------
+// Per-token INT8 activation quantization ("Inference Quantization ch.1" §9.2;
+// "Kimi 2.7 MoE, 4-bit storage to INT8" §3.3):
+//   s = max|x| / 127 (correctly rounded), q = clamp(rne(x / s), -127, 127),
+//   s == 0 -> divisor 1.
+// One CTA per source row; each thread holds CPT chunks of 8 bf16 in registers
+// (one 16-byte load each), so the row is read from HBM once.  With `dest`,
+// row m is written to the `dest_k` rows dest[m*dest_k + j] (the MoE dispatch
+// order) instead of row m.
+// ---------------------------------------------------------------------------
+constexpr int kQuantThreads = 256;
+
+template <int CPT>
+__global__ void __launch_bounds__(kQuantThreads) quant_act_kernel(
+    const uint16_t* __restrict__ X, int K, int ldx, int8_t* __restrict__ q, float* __restrict__ s_x,
+    int32_t* __restrict__ rowsum, int group, const int32_t* __restrict__ dest, int dest_k,
+    int32_t* status) {
+    const int m = blockIdx.x;
+    const int tid = threadIdx.x;
+    const int nchunk = K >> 3;
+    const uint4* xr = reinterpret_cast<const uint4*>(X + (size_t)m * ldx);
+
+    uint4 raw[CPT];
+    float amax = 0.0f;
+    uint32_t bad = 0;
+#pragma unroll
+    for (int i = 0; i < CPT; ++i) {
+        const int c = i * kQuantThreads + tid;
+        raw[i] = make_uint4(0, 0, 0, 0);
+        if (c < nchunk) {
+            raw[i] = __ldg(xr + c);
+            const uint32_t w[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                const uint32_t lo = w[h] & 0xFFFFu, hi = w[h] >> 16;
+                bad |= ((lo & 0x7F80u) == 0x7F80u) | ((hi & 0x7F80u) == 0x7F80u);
+                amax = fmaxf(amax, fabsf(bf16_bits_to_f32(lo)));
+                amax = fmaxf(amax, fabsf(bf16_bits_to_f32(hi)));
+            }
+        }
+    }
+    // block-wide max / or
+    __shared__ float red_max[kQuantThreads / 32];
+    __shared__ uint32_t red_bad[kQuantThreads / 32];
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
+        bad |= __shfl_xor_sync(0xFFFFFFFFu, bad, off);
+    }
+    if ((tid & 31) == 0) {
+        red_max[tid >> 5] = amax;
+        red_bad[tid >> 5] = bad;
+    }
+    __syncthreads();
+    amax = red_max[0];
+    bad = red_bad[0];
+#pragma unroll
+    for (int i = 1; i < kQuantThreads / 32; ++i) {
+        amax = fmaxf(amax, red_max[i]);
+        bad |= red_bad[i];
+    }
+    const float s = __fdiv_rn(amax, 127.0f);
+    const float d = (s > 0.0f) ? s : 1.0f;
+
+    const int nrows_out = dest ? dest_k : 1;
+#pragma unroll
+    for (int i = 0; i < CPT; ++i) {
+        const int c = i * kQuantThreads + tid;
+        const bool live = c < nchunk;
+        const uint32_t w[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
+        uint32_t packed[2] = {0u, 0u};
+        int32_t csum = 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const uint32_t bits = (e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xFFFFu);
+            float t = rintf(__fdiv_rn(bf16_bits_to_f32(bits), d));
+            t = fminf(fmaxf(t, -127.0f), 127.0f);
+            const int qi = (int)t;
+            csum += qi;
+            packed[e >> 2] |= ((uint32_t)(qi & 0xFF)) << (8 * (e & 3));
+        }
+        if (live) {
+            for (int j = 0; j < nrows_out; ++j) {
+                const int row = dest ? dest[(size_t)m * dest_k + j] : m;
+                *reinterpret_cast<uint2*>(q + (size_t)row * K + (size_t)c * 8) = make_uint2(packed[0], packed[1]);
+            }
+        }
+        if (rowsum) {
+            // group/8 consecutive chunks (8 or 16 lanes of one warp) form a
+            // group; chunks past the row end hold zeros.  All lanes shuffle.
+            const int lanes = group >> 3;
+            for (int off = lanes >> 1; off > 0; off >>= 1) csum += __shfl_xor_sync(0xFFFFFFFFu, csum, off);
+            if (live && (c % lanes) == 0) {
+                const int G = K / group;
+                for (int j = 0; j < nrows_out; ++j) {
+                    const int row = dest ? dest[(size_t)m * dest_k + j] : m;
+                    rowsum[(size_t)row * G + c / lanes] = csum;
+                }
+            }
+        }
+    }
+    if (tid == 0) {
+        for (int j = 0; j < nrows_out; ++j) {
+            const int row = dest ? dest[(size_t)m * dest_k + j] : m;
+            s_x[row] = s;
+        }
+        if (bad) report_status(status, kStatusNonfinite);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Offline group-wise 4-bit quantization and packing ("Quantization: formats,
+// error and the real execution path", sections "Basic mapping" and
+// "Symmetric group-wise reference"; "Inference Quantization ch.1" §6).
+// One thread per (output column n, group g); columns are consecutive across
+// the warp so every W load is coalesced.  Output layout: see w4a8.h.
+// ---------------------------------------------------------------------------
+template <int GROUP>
+__global__ void __launch_bounds__(128) pack_weights_kernel(const float* __restrict__ W, int K, int N,
+                                                           int symmetric, uint8_t* __restrict__ packed,
+                                                           float* __restrict__ s_w, uint8_t* __restrict__ z,
+                                                           int32_t* status) {
+    const int n = blockIdx.x * blockDim.x + threadIdx.x;
+    const int gi = blockIdx.y;
+    if (n >= N) return;
+    const int G = K / GROUP;
+    const float* col = W + (size_t)gi * GROUP * N + n;
+
+    float amax = 0.0f, lo = 0.0f, hi = 0.0f;
+    bool bad = false;
+    for (int k = 0; k < GROUP; ++k) {
+        const float w = __ldg(col + (size_t)k * N);
+        bad |= !isfinite(w);
+        amax = fmaxf(amax, fabsf(w));
+        lo = fminf(lo, w);
+        hi = fmaxf(hi, w);
+    }
+    float s, zf = 0.0f;
+    if (symmetric) {
+        s = __fdiv_rn(amax, 7.0f);
+    } else {
+        s = __fdiv_rn(__fsub_rn(hi, lo), 15.0f);
+    }
+    const float d = (s > 0.0f) ? s : 1.0f;
+    if (!symmetric) {
+        zf = rintf(__fdiv_rn(-lo, d));
+        zf = fminf(fmaxf(zf, 0.0f), 15.0f);
+    }
+
+    uint8_t* blk = packed + ((size_t)(n >> 6) * G + gi) * 32u * GROUP;
+    const int r = n & 63;
+#pragma unroll 1
+    for (int c = 0; c < GROUP / 32; ++c) {
+        uint32_t words[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+        for (int b = 0; b < 16; ++b) {
+            uint32_t nib2 = 0;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                const int k = 32 * c + 16 * half + b;
+                const float w = __ldg(col + (size_t)k * N);
+                float t = rintf(__fdiv_rn(w, d));
+                uint32_t code;
+                if (symmetric) {
+                    t = fminf(fmaxf(t, -7.0f), 7.0f);
+                    code = ((uint32_t)(int)t) & 0xFu;
+                } else {
+                    t = fminf(fmaxf(__fadd_rn(t, zf), 0.0f), 15.0f);
+                    code = (uint32_t)(int)t;
+                }
+                nib2 |= code << (4 * half);
+            }
+            words[b >> 2] |= nib2 << (8 * (b & 3));
+        }
+        *reinterpret_cast<uint4*>(blk + ((size_t)c * 64 + r) * 16) =
+            make_uint4(words[0], words[1], words[2], words[3]);
+    }
+    s_w[(size_t)gi * N + n] = s;
+    if (z) z[(size_t)gi * N + n] = (uint8_t)(int)zf;
+    if (bad) report_status(status, kStatusNonfinite);
+}
+
+// ---------------------------------------------------------------------------
+// MoE routing ("Kimi 2.7 MoE, 4-bit storage to INT8" §4.1, §4.4 step 1): the
+// router output stays fp32; top-k by logit (ties to the lower expert index);
+// weight = softmax over all E experts.  One warp per token; lane l holds
+// experts l, l+32, ...; the exp-sum uses a fixed reduction tree.
+// ---------------------------------------------------------------------------
+template <int EPL>
+__global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict__ logits, int T, int E,
+                                                         int topk, int32_t* __restrict__ idx,
+                                                         float* __restrict__ p, int32_t* status) {
+    const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (t >= T) return;
+    const float* l = logits + (size_t)t * E;
+    float v[EPL];
+    bool bad = false;
+    float mx = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+        const int e = i * 32 + lane;
+        v[i] = (e < E) ? __ldg(l + e) : -INFINITY;
+        if (e < E) {
+            bad |= !isfinite(v[i]);
+            mx = fmaxf(mx, v[i]);
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
+    float sum = 0.0f;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i)
+        if (i * 32 + lane < E) sum += expf(v[i] - mx);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, off);
+
+    uint32_t taken = 0;
+    for (int j = 0; j < topk; ++j) {
+        float bv = 0.0f;
+        int be = 0x7FFFFFFF;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+            const int e = i * 32 + lane;
+            if (e < E && !((taken >> i) & 1u) && (be == 0x7FFFFFFF || v[i] > bv)) {
+                bv = v[i];
+                be = e;
+            }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, off);
+            const int oe = __shfl_xor_sync(0xFFFFFFFFu, be, off);
+            if (oe != 0x7FFFFFFF && (be == 0x7FFFFFFF || ov > bv || (ov == bv && oe < be))) {
+                bv = ov;
+                be = oe;
+            }
+        }
+        if (be != 0x7FFFFFFF && lane == (be & 31)) taken |= 1u << (be >> 5);
+        if (lane == 0) {
+            idx[(size_t)t * topk + j] = (be == 0x7FFFFFFF) ? 0 : be;
+            p[(size_t)t * topk + j] = expf(bv - mx) / sum;
+        }
+    }
+    if (bad && lane == 0) report_status(status, kStatusNonfinite);
+}
+
+// ---------------------------------------------------------------------------
+// Dispatch ("Kimi 2.7 MoE, 4-bit storage to INT8" §4.4 step 3;
+// "Choosing a weight-quantization scheme", MoE grouped-GEMM path): count per
+// expert, exclusive prefix sum, then the stable (expert, token, slot) order.
+// Single CTA of 256 threads, deterministic (no order-dependent atomics):
+// tokens are walked in chunks of 256; inside a chunk, a per-(warp, expert)
+// lane bitmask gives each pair its rank among earlier tokens.  Also writes
+// the prefix over experts of ceil(count / BN) m-tiles for the grouped GEMMs.
+// ---------------------------------------------------------------------------
+constexpr int kDispatchThreads = 256;
+constexpr int kMaxExperts = 512;
+
+__global__ void __launch_bounds__(kDispatchThreads) dispatch_kernel(const int32_t* __restrict__ idx, int T,
+                                                                    int E, int topk, int bn,
+                                                                    int32_t* __restrict__ offsets,
+                                                                    int32_t* __restrict__ mtile_off,
+                                                                    int32_t* __restrict__ perm,
+                                                                    int32_t* __restrict__ inv) {
+    __shared__ int32_t cnt[kMaxExperts];
+    __shared__ int32_t base[kMaxExperts];
+    __shared__ uint32_t bits[kDispatchThreads / 32][kMaxExperts];
+    __shared__ int32_t wpre[kDispatchThreads / 32][kMaxExperts];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    for (int e = tid; e < E; e += kDispatchThreads) cnt[e] = 0;
+    __syncthreads();
+    const int pairs = T * topk;
+    for (int i = tid; i < pairs; i += kDispatchThreads) atomicAdd(&cnt[idx[i]], 1);
+    __syncthreads();
+    if (tid == 0) {
+        int32_t run = 0, tiles = 0;
+        for (int e = 0; e < E; ++e) {
+            offsets[e] = run;
+            mtile_off[e] = tiles;
+            base[e] = run;
+            run += cnt[e];
+            tiles += (cnt[e] + bn - 1) / bn;
+        }
+        offsets[E] = run;
+        mtile_off[E] = tiles;
+    }
+    __syncthreads();
+    for (int t0 = 0; t0 < T; t0 += kDispatchThreads) {
+        for (int e = lane; e < E; e += 32) bits[warp][e] = 0u;
+        __syncthreads();
+        const int t = t0 + tid;
+        if (t < T)
+            for (int j = 0; j < topk; ++j) atomicOr(&bits[warp][idx[(size_t)t * topk + j]], 1u << lane);
+        __syncthreads();
+        for (int e = tid; e < E; e += kDispatchThreads) {
+            int32_t run = 0;
+            for (int w = 0; w < kDispatchThreads / 32; ++w) {
+                wpre[w][e] = run;
+                run += __popc(bits[w][e]);
+            }
+            cnt[e] = run;  // chunk total for this expert
+        }
+        __syncthreads();
+        if (t < T) {
+            const uint32_t lt = (1u << lane) - 1u;
+            for (int j = 0; j < topk; ++j) {
+                const int e = idx[(size_t)t * topk + j];
+                const int32_t pos = base[e] + wpre[warp][e] + __popc(bits[warp][e] & lt);
+                inv[(size_t)t * topk + j] = pos;
+                perm[pos] = t * topk + j;
+            }
+        }
+        __syncthreads();
+        for (int e = tid; e < E; e += kDispatchThreads) base[e] += cnt[e];
+        __syncthreads();
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Weighted combine ("Kimi 2.7 MoE, 4-bit storage to INT8" §4.3-4.4 step 5):
+// out[t] = sum_j p[t,j] * y[inv(t,j)], fp32 in slot order, one bf16 rounding.
+// One thread per (token, 8 consecutive columns): 16-byte loads and stores.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict__ Yd,
+                                                      const float* __restrict__ p,
+                                                      const int32_t* __restrict__ inv, int T, int topk, int H,
+                                                      uint16_t* __restrict__ out) {
+    const int cpr = H >> 3;
+    const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (gid >= (long long)T * cpr) return;
+    const int t = (int)(gid / cpr), c = (int)(gid % cpr);
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
+    for (int j = 0; j < topk; ++j) {
+        const int r = __ldg(inv + (size_t)t * topk + j);
+        const float w = __ldg(p + (size_t)t * topk + j);
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(Yd + (size_t)r * H) + c);
+        const uint32_t ws[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const uint32_t bits = (e & 1) ? (ws[e >> 1] >> 16) : (ws[e >> 1] & 0xFFFFu);
+            acc[e] = fmaf(w, bf16_bits_to_f32(bits), acc[e]);
+        }
+    }
+    uint32_t o[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+        o[e] = (uint32_t)f32_to_bf16_bits(acc[2 * e]) | ((uint32_t)f32_to_bf16_bits(acc[2 * e + 1]) << 16);
+    *reinterpret_cast<uint4*>(out + (size_t)t * H + (size_t)c * 8) = make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// ---------------------------------------------------------------------------
+// Split-K finish: sums the fp32 partial tiles of each output tile in CTA
+// order (fixed, so the result does not depend on timing), applies s_x and
+// rounds to bf16.  Partial slot layout: [tile][slot][col BN][row 128].
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) splitk_finish_kernel(const float* __restrict__ part,
+                                                            const float* __restrict__ s_x, int M, int N, int G,
+                                                            int bn, int n_tiles, long long Q, int slots,
+                                                            uint16_t* __restrict__ Y, int ldy) {
+    const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (gid >= (long long)M * N) return;
+    const int m = (int)(gid / N), n = (int)(gid % N);
+    const long long t = (long long)(m / bn) * n_tiles + n / 128;
+    const long long u0 = t * G;
+    const long long c_first = u0 / Q, c_last = (u0 + G - 1) / Q;
+    float acc = 0.0f;
+    for (long long c = c_first; c <= c_last; ++c) {
+        const long long slot = c - c_first;
+        acc += __ldg(part + (((t * slots + slot) * bn + (m % bn)) * 128 + (n % 128)));
+    }
+    Y[(size_t)m * ldy + n] = f32_to_bf16_bits(__ldg(s_x + m) * acc);
+}
+
+// Test hook: one warp waits on a barrier nobody arrives on.
+__global__ void bounded_wait_selftest_kernel(int32_t* status, unsigned long long limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    WaitCtx w{&abort_flag, status, limit_ns};
+    if (threadIdx.x == 0) (void)wait_bounded(&bar, 0, w);
+    __syncthreads();
+}
+
+}  // namespace w4a8

@@ -1,0 +1,531 @@
+// libw4a8.so: the C ABI declared in include/w4a8.h.
+//
+// Host side only: argument / shape / descriptor checks, launch planning
+// (tile shape, persistent grid, split-K), TMA descriptor encoding, and the
+// launches.  Every call is asynchronous on the caller's stream and never
+// allocates; scratch lives in the caller's workspace.
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <mutex>
+
+#include "w4a8.h"
+#include "gemm_tc.cuh"
+#include "kernels_misc.cuh"
+
+using namespace w4a8;
+
+namespace {
+
+constexpr unsigned long long kDefaultWaitNs = 4000000000ull;  // 4 s per wait
+
+// ------------------------------------------------------------ device info --
+
+int sm_count_current() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    static std::atomic<int> cache[64];
+    if (dev >= 0 && dev < 64) {
+        int v = cache[dev].load();
+        if (v > 0) return v;
+    }
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    if (dev >= 0 && dev < 64) cache[dev].store(n);
+    return n;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// Tensor map over an int8 [rows][K] row-major matrix, box = group x bn,
+// swizzle = group bytes (64B or 128B).
+bool make_act_tmap(CUtensorMap* map, const void* base, int rows, int K, int group, int bn) {
+    EncodeTiledFn enc = get_encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)K};
+    cuuint32_t box[2] = {(cuuint32_t)group, (cuuint32_t)bn};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     group == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+w4a8_status last_cuda() { return cudaGetLastError() == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA; }
+
+// ---------------------------------------------------------- GEMM configs --
+
+template <int BN, int GROUP>
+struct Stages;
+template <> struct Stages<16, 128> { static constexpr int S = 12, SA = 3; };
+template <> struct Stages<32, 128> { static constexpr int S = 10, SA = 3; };
+template <> struct Stages<64, 128> { static constexpr int S = 8, SA = 3; };
+template <> struct Stages<128, 128> { static constexpr int S = 5, SA = 3; };
+template <> struct Stages<16, 64> { static constexpr int S = 16, SA = 4; };
+template <> struct Stages<32, 64> { static constexpr int S = 16, SA = 4; };
+template <> struct Stages<64, 64> { static constexpr int S = 12, SA = 4; };
+template <> struct Stages<128, 64> { static constexpr int S = 8, SA = 4; };
+
+template <int BN, int GROUP>
+w4a8_status launch_gemm_t(const CUtensorMap& tmap, const GemmParams& p, int grid, cudaStream_t stream) {
+    constexpr int S = Stages<BN, GROUP>::S, SA = Stages<BN, GROUP>::SA;
+    using C = GemmCfg<BN, GROUP, S, SA>;
+    auto kern = w4a8_gemm_tc_kernel<BN, GROUP, S, SA>;
+    static std::atomic<uint64_t> attr_done{0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const uint64_t bit = 1ull << (dev & 63);
+    if (!(attr_done.load() & bit)) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
+            return W4A8_ERR_CUDA;
+        attr_done.fetch_or(bit);
+    }
+    kern<<<grid, kGemmThreads, C::SMEM, stream>>>(tmap, p);
+    return last_cuda();
+}
+
+w4a8_status launch_gemm(int bn, int group, const CUtensorMap& tmap, const GemmParams& p, int grid,
+                        cudaStream_t stream) {
+    if (group == 128) {
+        switch (bn) {
+            case 16: return launch_gemm_t<16, 128>(tmap, p, grid, stream);
+            case 32: return launch_gemm_t<32, 128>(tmap, p, grid, stream);
+            case 64: return launch_gemm_t<64, 128>(tmap, p, grid, stream);
+            case 128: return launch_gemm_t<128, 128>(tmap, p, grid, stream);
+        }
+    } else {
+        switch (bn) {
+            case 16: return launch_gemm_t<16, 64>(tmap, p, grid, stream);
+            case 32: return launch_gemm_t<32, 64>(tmap, p, grid, stream);
+            case 64: return launch_gemm_t<64, 64>(tmap, p, grid, stream);
+            case 128: return launch_gemm_t<128, 64>(tmap, p, grid, stream);
+        }
+    }
+    return W4A8_ERR_UNSUPPORTED_SHAPE;
+}
+
+int pick_bn(long long rows_per_group) {
+    if (rows_per_group <= 16) return 16;
+    if (rows_per_group <= 32) return 32;
+    if (rows_per_group <= 64) return 64;
+    return 128;
+}
+
+// Launch plan of the plain (dense) GEMM.
+struct GemmPlan {
+    int bn, m_tiles, n_tiles, G, grid, slots;
+    long long Q;
+    bool splitk;
+    size_t ws_bytes;
+};
+
+GemmPlan plan_gemm(int M, int N, int K, int group, int sms) {
+    GemmPlan pl{};
+    pl.bn = pick_bn(M);
+    pl.m_tiles = (M + pl.bn - 1) / pl.bn;
+    pl.n_tiles = (N + 127) / 128;
+    pl.G = K / group;
+    const long long tiles = (long long)pl.m_tiles * pl.n_tiles;
+    const long long U = tiles * pl.G;
+    if (sms <= 0) sms = 1;
+    const long long waves = (tiles + sms - 1) / sms;
+    const double eff = (double)tiles / (double)(waves * sms);
+    pl.splitk = (eff < 0.85) && pl.G > 1;
+    if (pl.splitk) {
+        pl.Q = (U + sms - 1) / sms;
+        pl.grid = (int)((U + pl.Q - 1) / pl.Q);
+        pl.slots = (int)((pl.G + pl.Q - 1) / pl.Q) + 1;
+        pl.ws_bytes = (size_t)tiles * pl.slots * pl.bn * 128 * sizeof(float);
+    } else {
+        pl.Q = (long long)pl.G * waves;
+        pl.grid = (int)((tiles + waves - 1) / waves);
+        pl.slots = 0;
+        pl.ws_bytes = 0;
+    }
+    return pl;
+}
+
+w4a8_status check_wdesc(const w4a8_wdesc* w) {
+    if (!w) return W4A8_ERR_INVALID_ARG;
+    if (w->bits != 4 || w->layout_version != W4A8_LAYOUT_VERSION) return W4A8_ERR_FORMAT_MISMATCH;
+    if (w->group != 64 && w->group != 128) return W4A8_ERR_FORMAT_MISMATCH;
+    if (w->symmetric != 0 && w->symmetric != 1) return W4A8_ERR_FORMAT_MISMATCH;
+    if (w->K <= 0 || w->N <= 0 || w->K % w->group != 0 || w->N % 64 != 0) return W4A8_ERR_FORMAT_MISMATCH;
+    return W4A8_OK;
+}
+
+w4a8_status gemm_impl(const int8_t* qx, const float* s_x, const uint8_t* packed, const float* s_w,
+                      const uint8_t* z, const w4a8_wdesc* w, int M, uint16_t* Y, int ldy, int32_t* P,
+                      void* workspace, size_t ws_bytes, int32_t* dev_status, void* stream) {
+    w4a8_status st = check_wdesc(w);
+    if (st != W4A8_OK) return st;
+    if (M < 0 || !Y || ldy < w->N) return W4A8_ERR_INVALID_ARG;
+    if (M == 0) return W4A8_OK;
+    if (!qx || !s_x || !packed || !s_w) return W4A8_ERR_INVALID_ARG;
+    if (w->symmetric ? (z != nullptr) : (z == nullptr)) return W4A8_ERR_FORMAT_MISMATCH;
+    if (!aligned16(qx) || !aligned16(packed) || (z && !aligned16(z))) return W4A8_ERR_INVALID_ARG;
+    if (w->K % 16 != 0 || w->K > (1 << 24) || M > (1 << 24)) return W4A8_ERR_UNSUPPORTED_SHAPE;
+    const GemmPlan pl = plan_gemm(M, w->N, w->K, w->group, sm_count_current());
+    if (pl.ws_bytes > 0 && (!workspace || ws_bytes < pl.ws_bytes)) return W4A8_ERR_WORKSPACE;
+
+    CUtensorMap tmap;
+    if (!make_act_tmap(&tmap, qx, M, w->K, w->group, pl.bn)) return W4A8_ERR_CUDA;
+    GemmParams p{};
+    p.packed = packed;
+    p.s_w = s_w;
+    p.z = z;
+    p.N = w->N;
+    p.K = w->K;
+    p.G = pl.G;
+    p.symmetric = w->symmetric;
+    p.s_x = s_x;
+    p.M = M;
+    p.mode = pl.splitk ? kModeSplitK : kModePlain;
+    p.Y = Y;
+    p.ldy = ldy;
+    p.partial = static_cast<float*>(workspace);
+    p.slots = pl.slots;
+    p.dbgP = P;
+    p.n_tiles = pl.n_tiles;
+    p.m_tiles = pl.m_tiles;
+    p.units_per_cta = pl.Q;
+    p.status = dev_status;
+    p.wait_ns = kDefaultWaitNs;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    st = launch_gemm(pl.bn, w->group, tmap, p, pl.grid, s);
+    if (st != W4A8_OK) return st;
+    if (pl.splitk) {
+        const long long n = (long long)M * w->N;
+        splitk_finish_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(
+            static_cast<const float*>(workspace), s_x, M, w->N, pl.G, pl.bn, pl.n_tiles, pl.Q, pl.slots, Y, ldy);
+        st = last_cuda();
+    }
+    return st;
+}
+
+w4a8_status launch_quant(const uint16_t* X, int rows, int K, int ldx, int8_t* q, float* s_x, int32_t* rowsum,
+                         int group, const int32_t* dest, int dest_k, int32_t* status, cudaStream_t s) {
+    if (rows == 0) return W4A8_OK;
+    const int cpt = (K / 8 + kQuantThreads - 1) / kQuantThreads;
+    switch (cpt) {
+        case 1: quant_act_kernel<1><<<rows, kQuantThreads, 0, s>>>(X, K, ldx, q, s_x, rowsum, group, dest, dest_k, status); break;
+        case 2: quant_act_kernel<2><<<rows, kQuantThreads, 0, s>>>(X, K, ldx, q, s_x, rowsum, group, dest, dest_k, status); break;
+        case 3: quant_act_kernel<3><<<rows, kQuantThreads, 0, s>>>(X, K, ldx, q, s_x, rowsum, group, dest, dest_k, status); break;
+        case 4: quant_act_kernel<4><<<rows, kQuantThreads, 0, s>>>(X, K, ldx, q, s_x, rowsum, group, dest, dest_k, status); break;
+        default: return W4A8_ERR_UNSUPPORTED_SHAPE;
+    }
+    return last_cuda();
+}
+
+// ------------------------------------------------------------ MoE layout --
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+struct MoeLayout {
+    size_t mtile_off, perm, inv, qx, sx, h, qh, sh, yd, total;
+};
+
+MoeLayout moe_layout(int T, int E, int topk, int H, int I) {
+    MoeLayout L{};
+    const size_t R = (size_t)T * topk;
+    size_t o = 0;
+    L.mtile_off = o; o = align_up(o + sizeof(int32_t) * (E + 1), 256);
+    L.perm = o;      o = align_up(o + sizeof(int32_t) * R, 256);
+    L.inv = o;       o = align_up(o + sizeof(int32_t) * R, 256);
+    L.qx = o;        o = align_up(o + R * H, 256);
+    L.sx = o;        o = align_up(o + sizeof(float) * R, 256);
+    L.h = o;         o = align_up(o + 2 * R * I, 256);
+    L.qh = o;        o = align_up(o + R * I, 256);
+    L.sh = o;        o = align_up(o + sizeof(float) * R, 256);
+    L.yd = o;        o = align_up(o + 2 * R * H, 256);
+    L.total = o;
+    return L;
+}
+
+w4a8_status check_moe(int T, int E, int topk, const w4a8_wdesc* w1, const w4a8_wdesc* w2) {
+    w4a8_status st = check_wdesc(w1);
+    if (st != W4A8_OK) return st;
+    st = check_wdesc(w2);
+    if (st != W4A8_OK) return st;
+    if (T < 0 || E <= 0 || topk <= 0 || topk > E) return W4A8_ERR_INVALID_ARG;
+    if (w1->symmetric != w2->symmetric || w1->group != w2->group) return W4A8_ERR_FORMAT_MISMATCH;
+    const int H = w1->K, I2 = w1->N;
+    if (I2 % 2 != 0 || w2->K != I2 / 2 || w2->N != H) return W4A8_ERR_FORMAT_MISMATCH;
+    const int I = I2 / 2;
+    if (E > kMaxExperts || topk > 16) return W4A8_ERR_UNSUPPORTED_SHAPE;
+    if (H % 64 != 0 || I % 64 != 0 || H > 8192 || I > 8192) return W4A8_ERR_UNSUPPORTED_SHAPE;
+    if ((long long)T * topk > (1ll << 26)) return W4A8_ERR_UNSUPPORTED_SHAPE;
+    return W4A8_OK;
+}
+
+}  // namespace
+
+// ===================================================================== ABI ==
+
+extern "C" {
+
+int w4a8_abi_version(void) { return W4A8_ABI_VERSION; }
+
+const char* w4a8_status_string(w4a8_status s) {
+    switch (s) {
+        case W4A8_OK: return "W4A8_OK";
+        case W4A8_ERR_INVALID_ARG: return "W4A8_ERR_INVALID_ARG";
+        case W4A8_ERR_UNSUPPORTED_SHAPE: return "W4A8_ERR_UNSUPPORTED_SHAPE";
+        case W4A8_ERR_FORMAT_MISMATCH: return "W4A8_ERR_FORMAT_MISMATCH";
+        case W4A8_ERR_NONFINITE: return "W4A8_ERR_NONFINITE";
+        case W4A8_ERR_TIMEOUT: return "W4A8_ERR_TIMEOUT";
+        case W4A8_ERR_CUDA: return "W4A8_ERR_CUDA";
+        case W4A8_ERR_WORKSPACE: return "W4A8_ERR_WORKSPACE";
+    }
+    return "W4A8_ERR_UNKNOWN";
+}
+
+size_t w4a8_packed_bytes(int K, int N) {
+    if (K <= 0 || N <= 0) return 0;
+    return (size_t)K * (size_t)N / 2;
+}
+
+size_t w4a8_gemm_workspace_size(int M, const w4a8_wdesc* w) {
+    if (M <= 0 || check_wdesc(w) != W4A8_OK) return 0;
+    return plan_gemm(M, w->N, w->K, w->group, sm_count_current()).ws_bytes;
+}
+
+size_t w4a8_moe_workspace_size(int T, int E, int topk, const w4a8_wdesc* w1, const w4a8_wdesc* w2) {
+    if (check_moe(T, E, topk, w1, w2) != W4A8_OK) return 0;
+    return moe_layout(T, E, topk, w1->K, w1->N / 2).total;
+}
+
+w4a8_status w4a8_moe_workspace_layout(int T, int E, int topk, const w4a8_wdesc* w1, const w4a8_wdesc* w2,
+                                      w4a8_moe_ws_layout* out) {
+    w4a8_status st = check_moe(T, E, topk, w1, w2);
+    if (st != W4A8_OK) return st;
+    if (!out) return W4A8_ERR_INVALID_ARG;
+    const MoeLayout L = moe_layout(T, E, topk, w1->K, w1->N / 2);
+    out->perm = L.perm;
+    out->inv = L.inv;
+    out->qx = L.qx;
+    out->sx = L.sx;
+    out->h = L.h;
+    out->qh = L.qh;
+    out->sh = L.sh;
+    out->yd = L.yd;
+    out->total = L.total;
+    return W4A8_OK;
+}
+
+w4a8_status w4a8_pack_weights(const float* W, int K, int N, int group, int symmetric, uint8_t* packed,
+                              float* s_w, uint8_t* z, w4a8_wdesc* out, int32_t* dev_status, void* stream) {
+    if (!W || !packed || !s_w) return W4A8_ERR_INVALID_ARG;
+    if (group != 64 && group != 128) return W4A8_ERR_INVALID_ARG;
+    if (symmetric != 0 && symmetric != 1) return W4A8_ERR_INVALID_ARG;
+    if (K <= 0 || N <= 0 || K % group != 0 || N % 64 != 0) return W4A8_ERR_INVALID_ARG;
+    if (symmetric ? (z != nullptr) : (z == nullptr)) return W4A8_ERR_INVALID_ARG;
+    if (!aligned16(packed)) return W4A8_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    dim3 grid((N + 127) / 128, K / group);
+    if (group == 128)
+        pack_weights_kernel<128><<<grid, 128, 0, s>>>(W, K, N, symmetric, packed, s_w, z, dev_status);
+    else
+        pack_weights_kernel<64><<<grid, 128, 0, s>>>(W, K, N, symmetric, packed, s_w, z, dev_status);
+    w4a8_status st = last_cuda();
+    if (st == W4A8_OK && out) {
+        out->bits = 4;
+        out->symmetric = symmetric;
+        out->group = group;
+        out->K = K;
+        out->N = N;
+        out->layout_version = W4A8_LAYOUT_VERSION;
+    }
+    return st;
+}
+
+w4a8_status w4a8_quant_act(const uint16_t* X, int M, int K, int ldx, int group_for_rowsum, int8_t* qx,
+                           float* s_x, int32_t* rowsum, int32_t* dev_status, void* stream) {
+    if (M < 0 || K <= 0 || ldx < K) return W4A8_ERR_INVALID_ARG;
+    if (M == 0) return W4A8_OK;
+    if (!X || !qx || !s_x) return W4A8_ERR_INVALID_ARG;
+    if (K % 8 != 0 || ldx % 8 != 0 || !aligned16(X)) return W4A8_ERR_UNSUPPORTED_SHAPE;
+    if (K > 8192) return W4A8_ERR_UNSUPPORTED_SHAPE;
+    if (rowsum) {
+        if (group_for_rowsum != 64 && group_for_rowsum != 128) return W4A8_ERR_INVALID_ARG;
+        if (K % group_for_rowsum != 0) return W4A8_ERR_INVALID_ARG;
+    } else if (group_for_rowsum != 0) {
+        return W4A8_ERR_INVALID_ARG;
+    }
+    if ((reinterpret_cast<uintptr_t>(qx) & 7u) != 0 || K % 8 != 0) return W4A8_ERR_UNSUPPORTED_SHAPE;
+    return launch_quant(X, M, K, ldx, qx, s_x, rowsum, group_for_rowsum, nullptr, 0, dev_status,
+                        static_cast<cudaStream_t>(stream));
+}
+
+w4a8_status w4a8_gemm(const int8_t* qx, const float* s_x, const uint8_t* packed, const float* s_w, const uint8_t* z,
+                      const w4a8_wdesc* w, int M, uint16_t* Y, int ldy, void* workspace, size_t ws_bytes,
+                      int32_t* dev_status, void* stream) {
+    return gemm_impl(qx, s_x, packed, s_w, z, w, M, Y, ldy, nullptr, workspace, ws_bytes, dev_status, stream);
+}
+
+w4a8_status w4a8_gemm_debug_partials(const int8_t* qx, const float* s_x, const uint8_t* packed, const float* s_w,
+                                     const uint8_t* z, const w4a8_wdesc* w, int M, uint16_t* Y, int ldy, int32_t* P,
+                                     void* workspace, size_t ws_bytes, int32_t* dev_status, void* stream) {
+    if (!P) return W4A8_ERR_INVALID_ARG;
+    return gemm_impl(qx, s_x, packed, s_w, z, w, M, Y, ldy, P, workspace, ws_bytes, dev_status, stream);
+}
+
+w4a8_status w4a8_moe_grouped_gemm(const uint16_t* X, const float* logits, int T, int E, int topk,
+                                  const uint8_t* w1_packed, const float* w1_s, const uint8_t* w1_z,
+                                  const w4a8_wdesc* w1, const uint8_t* w2_packed, const float* w2_s,
+                                  const uint8_t* w2_z, const w4a8_wdesc* w2, uint16_t* out,
+                                  int32_t* topk_idx_out, float* topk_w_out, int32_t* expert_offsets_out,
+                                  void* workspace, size_t ws_bytes, int32_t* dev_status, void* stream) {
+    w4a8_status st = check_moe(T, E, topk, w1, w2);
+    if (st != W4A8_OK) return st;
+    if (T == 0) return W4A8_OK;
+    if (!X || !logits || !w1_packed || !w1_s || !w2_packed || !w2_s || !out || !topk_idx_out || !topk_w_out ||
+        !expert_offsets_out)
+        return W4A8_ERR_INVALID_ARG;
+    const bool sym = w1->symmetric != 0;
+    if (sym ? (w1_z || w2_z) : (!w1_z || !w2_z)) return W4A8_ERR_FORMAT_MISMATCH;
+    if (!aligned16(X) || !aligned16(out) || !aligned16(w1_packed) || !aligned16(w2_packed) ||
+        (w1_z && !aligned16(w1_z)) || (w2_z && !aligned16(w2_z)))
+        return W4A8_ERR_INVALID_ARG;
+    const int H = w1->K, I = w1->N / 2, group = w1->group;
+    const MoeLayout L = moe_layout(T, E, topk, H, I);
+    if (!workspace || ws_bytes < L.total || !aligned16(workspace)) return W4A8_ERR_WORKSPACE;
+    const int sms = sm_count_current();
+    if (sms <= 0) return W4A8_ERR_CUDA;
+
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    int32_t* mtile_off = reinterpret_cast<int32_t*>(ws + L.mtile_off);
+    int32_t* perm = reinterpret_cast<int32_t*>(ws + L.perm);
+    int32_t* inv = reinterpret_cast<int32_t*>(ws + L.inv);
+    int8_t* qx = reinterpret_cast<int8_t*>(ws + L.qx);
+    float* sx = reinterpret_cast<float*>(ws + L.sx);
+    uint16_t* h = reinterpret_cast<uint16_t*>(ws + L.h);
+    int8_t* qh = reinterpret_cast<int8_t*>(ws + L.qh);
+    float* sh = reinterpret_cast<float*>(ws + L.sh);
+    uint16_t* yd = reinterpret_cast<uint16_t*>(ws + L.yd);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int R = T * topk;
+    const int bn = pick_bn(((long long)R + E - 1) / E);
+
+    // 1. routing
+    {
+        const int epl = (E + 31) / 32;
+        const unsigned blocks = (unsigned)(((long long)T * 32 + 255) / 256);
+        switch (epl) {
+#define W4A8_ROUTE(n) case n: route_topk_kernel<n><<<blocks, 256, 0, s>>>(logits, T, E, topk, topk_idx_out, topk_w_out, dev_status); break;
+            W4A8_ROUTE(1) W4A8_ROUTE(2) W4A8_ROUTE(3) W4A8_ROUTE(4) W4A8_ROUTE(5) W4A8_ROUTE(6) W4A8_ROUTE(7)
+            W4A8_ROUTE(8) W4A8_ROUTE(9) W4A8_ROUTE(10) W4A8_ROUTE(11) W4A8_ROUTE(12) W4A8_ROUTE(13)
+            W4A8_ROUTE(14) W4A8_ROUTE(15) W4A8_ROUTE(16)
+#undef W4A8_ROUTE
+            default: return W4A8_ERR_UNSUPPORTED_SHAPE;
+        }
+        if ((st = last_cuda()) != W4A8_OK) return st;
+    }
+    // 2. dispatch
+    dispatch_kernel<<<1, kDispatchThreads, 0, s>>>(topk_idx_out, T, E, topk, bn, expert_offsets_out, mtile_off,
+                                                   perm, inv);
+    if ((st = last_cuda()) != W4A8_OK) return st;
+    // 3. quantize X straight into dispatch order
+    if ((st = launch_quant(X, T, H, H, qx, sx, nullptr, 0, inv, topk, dev_status, s)) != W4A8_OK) return st;
+    // 4. gate_up + SiLU * up
+    {
+        CUtensorMap tmap;
+        if (!make_act_tmap(&tmap, qx, R, H, group, bn)) return W4A8_ERR_CUDA;
+        GemmParams p{};
+        p.packed = w1_packed;
+        p.s_w = w1_s;
+        p.z = w1_z;
+        p.N = w1->N;
+        p.K = H;
+        p.G = H / group;
+        p.packed_estride = (long long)w1->N * H / 2;
+        p.sw_estride = (long long)p.G * w1->N;
+        p.symmetric = w1->symmetric;
+        p.s_x = sx;
+        p.mode = kModeGateUp;
+        p.Y = h;
+        p.ldy = I;
+        p.n_tiles = I / 64;
+        p.expert_off = expert_offsets_out;
+        p.mtile_off = mtile_off;
+        p.E = E;
+        p.I = I;
+        p.status = dev_status;
+        p.wait_ns = kDefaultWaitNs;
+        if ((st = launch_gemm(bn, group, tmap, p, sms, s)) != W4A8_OK) return st;
+    }
+    // 5. quantize h per (token, expert) row
+    if ((st = launch_quant(h, R, I, I, qh, sh, nullptr, 0, nullptr, 0, dev_status, s)) != W4A8_OK) return st;
+    // 6. down
+    {
+        CUtensorMap tmap;
+        if (!make_act_tmap(&tmap, qh, R, I, group, bn)) return W4A8_ERR_CUDA;
+        GemmParams p{};
+        p.packed = w2_packed;
+        p.s_w = w2_s;
+        p.z = w2_z;
+        p.N = H;
+        p.K = I;
+        p.G = I / group;
+        p.packed_estride = (long long)H * I / 2;
+        p.sw_estride = (long long)p.G * H;
+        p.symmetric = w2->symmetric;
+        p.s_x = sh;
+        p.mode = kModeDown;
+        p.Y = yd;
+        p.ldy = H;
+        p.n_tiles = (H + 127) / 128;
+        p.expert_off = expert_offsets_out;
+        p.mtile_off = mtile_off;
+        p.E = E;
+        p.status = dev_status;
+        p.wait_ns = kDefaultWaitNs;
+        if ((st = launch_gemm(bn, group, tmap, p, sms, s)) != W4A8_OK) return st;
+    }
+    // 7. weighted combine
+    {
+        const long long n = (long long)T * (H / 8);
+        combine_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(yd, topk_w_out, inv, T, topk, H, out);
+        if ((st = last_cuda()) != W4A8_OK) return st;
+    }
+    return W4A8_OK;
+}
+
+w4a8_status w4a8_get_device_status(const int32_t* dev_status, void* stream) {
+    if (!dev_status) return W4A8_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return W4A8_ERR_CUDA;
+    int32_t v = 0;
+    if (cudaMemcpy(&v, dev_status, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) return W4A8_ERR_CUDA;
+    return static_cast<w4a8_status>(v);
+}
+
+w4a8_status w4a8_selftest_bounded_wait(int32_t* dev_status, uint64_t limit_ns, void* stream) {
+    if (!dev_status || limit_ns < 1000ull || limit_ns > 1000000000ull) return W4A8_ERR_INVALID_ARG;
+    bounded_wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(dev_status, limit_ns);
+    return last_cuda();
+}
+
+}  // extern "C"
