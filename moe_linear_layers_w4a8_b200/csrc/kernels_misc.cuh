@@ -263,7 +263,7 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
             p[(size_t)t * topk + j] = expf(bv - mx) / sum;
         }
     }
-    if (bad && lane == 0) report_status(status, kStatusNonfinite);
+    if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) report_status(status, kStatusNonfinite);
 }
 
 // ---------------------------------------------------------------------------
