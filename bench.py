@@ -1,0 +1,647 @@
+"""Benchmark of the W4A8 Linear / MoE-expert path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload decode|prefill|moe_sym|moe_asym_decode|moe_asym_prefill]
+                    [--m M]
+
+One "step" is one pass of the hot path over one batch of synthetic input:
+  decode / prefill:  per-token INT8 quantization of X, then the W4A8 GEMM;
+  moe_*:             the whole MoE layer (route, dispatch + quantize, grouped
+                     gate_up with SiLU*up, quantize h, grouped down, combine).
+The default workload is the decode-shaped linear (M=32, K=4096, N=14336,
+symmetric int4 group 128, 8 outlier channels x50), whose metric is the
+weight bytes streamed per second.
+
+Timing: W untimed warm-up steps, then exactly K steps, each bracketed by a
+barrier + synchronize, timed with CUDA events on the launching stream (max
+over ranks).  The steps run as CUDA-graph replays; packed weights are
+rotated over enough copies that every step reads them from HBM, not L2.
+The dominant kernel's per-launch time is measured with CUDA events around
+its launches in the last graph replay of the timed region.  SM clocks and
+throttle reasons are sampled through NVML during the timed region.
+
+`e2e` repeats the metric through the public API call a user makes, with the
+step's input copied host->device from pinned memory and the result read back
+device->host inside the timed region.
+
+`--impl reference` times the CPU oracle (test infrastructure, the only
+reference this path has) on a bounded sample of the same workload.
+Multi-GPU (torchrun): every rank runs an independent replica of the workload
+(the path has no exchange step); value = all ranks' work / max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "W4A8 GEMM TOPS (prefill) & weight GB/s (decode) vs B200 roofline; MoE tokens/s"
+L2_BYTES = 126 * 1024 * 1024
+
+DEFAULT_STEPS = {"decode": 20000, "prefill": 1500, "moe_sym": 2000, "moe_asym_decode": 400,
+                 "moe_asym_prefill": 200}
+
+
+# ---------------------------------------------------------------- peaks ---
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                    bf16_sus=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), source="measured")
+    except Exception:
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, source="fallback")
+
+
+# --------------------------------------------------------------- clocks ---
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML in a thread."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, index: int):
+        self.ok = False
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            pass
+        self._stop = threading.Event()
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= int(self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+            except Exception:
+                pass
+            time.sleep(0.005)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+            if not self.samples:  # region shorter than one period: take one sample now
+                try:
+                    self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                    self.reasons |= int(self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+                except Exception:
+                    pass
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"], "samples": 0}
+        names = [n for b, n in self.REASONS.items() if self.reasons & b and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------ workloads ---
+
+class LinearWorkload:
+    """Per-token INT8 quant + W4A8 GEMM on a [M, K] x [K, N] linear."""
+
+    def __init__(self, name, M, K=4096, N=14336, group=128, device="cuda"):
+        self.name, self.M, self.K, self.N, self.group = name, M, K, N, group
+        self.dev = device
+        self.decode = name == "decode"
+
+    def setup(self):
+        import torch
+        import moe_linear_layers_w4a8_b200 as m
+        from synth import gen_linear
+        self.m = m
+        M, K, N, g = self.M, self.K, self.N, self.group
+        inp = gen_linear(M, K, N, seed=0, n_outliers=8, outlier_scale=50.0)
+        self.X_host = inp.X
+        pw = m.w4a8_pack_weights(inp.W.to(self.dev), g, True)
+        self.w_bytes = N * K // 2 + (K // g) * N * 4
+        # enough weight copies that the weights of consecutive steps are not in L2
+        self.copies = [pw]
+        if self.decode:
+            n = max(2, math.ceil(2 * L2_BYTES / self.w_bytes) + 1)
+            for _ in range(n - 1):
+                self.copies.append(m.PackedWeight(pw.packed.clone(), pw.s_w.clone(), None, pw.desc.copy()))
+        self.X = inp.X.to(self.dev)
+        self.q = torch.empty(M, K, dtype=torch.int8, device=self.dev)
+        self.s = torch.empty(M, dtype=torch.float32, device=self.dev)
+        self.Y = torch.empty(M, N, dtype=torch.bfloat16, device=self.dev)
+        ws = m.w4a8_gemm_workspace_size(M, pw)
+        self.ws = torch.empty(max(ws, 16), dtype=torch.uint8, device=self.dev)
+        self.splitk = ws > 0
+        self.launches_per_step = 3 if self.splitk else 2
+
+    def step(self, i, ev=None):
+        m = self.m
+        m.w4a8_quant_act(self.X, q_out=self.q, s_out=self.s)
+        if ev is not None:
+            ev[0].record()
+        m.w4a8_gemm(self.q, self.s, self.copies[i % len(self.copies)], out=self.Y, workspace=self.ws)
+        if ev is not None:
+            ev[1].record()
+
+    # metric
+    def units(self):
+        if self.decode:
+            return self.w_bytes / 1e9, "GB/s", "weight+scale bytes streamed per second"
+        return 2.0 * self.M * self.N * self.K / 1e12, "TOPS", "2*M*N*K int8 ops per second"
+
+    def kernel_roofline(self, peaks):
+        M, K, N, g = self.M, self.K, self.N, self.group
+        if self.decode:
+            alg = N * K // 2 + (K // g) * N * 4 + M * K + 4 * M + 2 * M * N
+            return dict(bound="hbm", per_launch=alg, unit="GB/s", scale=1e9, peak=peaks["hbm"],
+                        peak_note=f"hbm_gbs ({peaks['source']})")
+        ops = 2.0 * M * N * K
+        return dict(bound="tensor", per_launch=ops, unit="TOPS", scale=1e12, peak=2.0 * peaks["bf16_sus"],
+                    peak_note=f"2 x bf16_tflops_sustained ({peaks['source']}; int8/bf16 nominal ratio 2)")
+
+    def config(self):
+        base = {"workload": f"{self.name} linear M={self.M} K={self.K} N={self.N} symmetric int4 g={self.group}",
+                "M": self.M, "K": self.K, "N": self.N, "group": self.group}
+        if not hasattr(self, "copies"):
+            return base
+        return dict(base, **{
+                "l2": (f"{len(self.copies)} packed-weight copies rotated "
+                       f"({len(self.copies) * self.w_bytes / 2**20:.0f} MiB > 2x L2)" if self.decode else
+                       "per-step activations+output "
+                       f"{(self.M * self.K * 3 + 2 * self.M * self.N) / 2**20:.0f} MiB > L2"),
+                "schedule": "split-K" if self.splitk else "data-parallel tiles"})
+
+    def e2e_setup(self):
+        import torch
+        self.X_pin = self.X_host.pin_memory()
+        self.Y_pin = torch.empty(self.M, self.N, dtype=torch.bfloat16).pin_memory()
+        self.X_dev2 = torch.empty_like(self.X)
+        return self.X_pin.numel() * 2, self.Y_pin.numel() * 2
+
+    def e2e_step(self, i):
+        self.X_dev2.copy_(self.X_pin, non_blocking=True)
+        Y = self.m.w4a8_linear(self.X_dev2, self.copies[i % len(self.copies)], out=self.Y, workspace=self.ws,
+                               q_buf=self.q, s_buf=self.s)
+        self.Y_pin.copy_(Y, non_blocking=True)
+
+    # CPU oracle on a bounded sample of the same workload
+    def oracle_step_setup(self, n_cols):
+        import numpy as np
+        import oracle as O
+        import torch
+        W = self._W_host()
+        cols = np.sort(np.random.default_rng(0).choice(self.N, n_cols, replace=False))
+        codes, s, _, _ = O.quant_weights(W[:, cols].copy(), self.group, True)  # offline step, untimed
+        self._orc = (O, codes, s, self.X_host.view(torch.int16).numpy().view(np.uint16))
+        return n_cols / self.N
+
+    def _W_host(self):
+        from synth import gen_linear
+        return gen_linear(self.M, self.K, self.N, seed=0, n_outliers=8, outlier_scale=50.0).W.numpy()
+
+    def oracle_step(self):
+        O, codes, s, Xb = self._orc
+        O.linear(Xb, codes, s, None, self.group)
+
+
+class MoEWorkload:
+    """One MoE expert layer."""
+
+    def __init__(self, name, device="cuda"):
+        from synth import CONFIGS
+        c = CONFIGS[name]
+        self.name = name
+        self.T, self.H, self.E, self.topk, self.I = c["T"], c["H"], c["E"], c["topk"], c["I"]
+        self.group, self.sym, self.zipf, self.wp = c["group"], c["symmetric"], c["zipf"], c["w_outlier_p"]
+        self.dev = device
+        self.launches_per_step = 7
+
+    def _weight(self, e, which, device):
+        from synth import gen_expert_weight
+        K, N = (self.H, 2 * self.I) if which == 0 else (self.I, self.H)
+        return gen_expert_weight(0, e, which, K, N, outlier_p=self.wp, device=device)
+
+    def setup(self):
+        import torch
+        import moe_linear_layers_w4a8_b200 as m
+        from synth import gen_moe_activations
+        self.m = m
+        inp = gen_moe_activations(self.T, self.H, self.E, seed=0, zipf=self.zipf)
+        self.X_host, self.L_host = inp.X, inp.logits
+        self.X, self.L = inp.X.to(self.dev), inp.logits.to(self.dev)
+        self.w1 = m.w4a8_pack_expert_weights(lambda e: self._weight(e, 0, self.dev), self.E, self.H, 2 * self.I,
+                                             self.group, self.sym, self.dev)
+        self.w2 = m.w4a8_pack_expert_weights(lambda e: self._weight(e, 1, self.dev), self.E, self.I, self.H,
+                                             self.group, self.sym, self.dev)
+        ws = m.w4a8_moe_workspace_size(self.T, self.E, self.topk, self.w1, self.w2)
+        self.ws = torch.empty(ws, dtype=torch.uint8, device=self.dev)
+        self.out = torch.empty(self.T, self.H, dtype=torch.bfloat16, device=self.dev)
+        # Expert hit count, for the bytes of the weight-streaming roofline.
+        r = m.w4a8_moe_grouped_gemm(self.X, self.L, self.topk, self.w1, self.w2, workspace=self.ws, out=self.out)
+        offs = r["expert_offsets"].cpu()
+        self.hit = int(((offs[1:] - offs[:-1]) > 0).sum())
+        self.counts = (offs[1:] - offs[:-1]).tolist()
+
+    STAGES = ["route", "dispatch", "quant_x", "gate_up", "quant_h", "down", "combine"]
+
+    def step(self, i, ev=None):
+        self.m.w4a8_moe_grouped_gemm(self.X, self.L, self.topk, self.w1, self.w2, workspace=self.ws, out=self.out,
+                                     stage_events=ev)
+
+    def units(self):
+        return self.T / 1e6, "Mtokens/s", "tokens per second through the whole layer"
+
+    def kernel_roofline(self, peaks):
+        H, I, g, R = self.H, self.I, self.group, self.T * self.topk
+        zb = 0 if self.sym else 1
+        # the gate_up GEMM is the largest launch of the layer
+        w1_expert = H * 2 * I // 2 + (H // g) * 2 * I * (4 + zb)
+        act = R * H + 4 * R + R * I * 2  # q_x rows in, h rows out
+        ops = 2.0 * R * H * 2 * I
+        if self.name == "moe_asym_decode":
+            return dict(bound="hbm", per_launch=self.hit * w1_expert + act, unit="GB/s", scale=1e9,
+                        peak=peaks["hbm"], kernel="gate_up",
+                        peak_note=f"hbm_gbs ({peaks['source']}); gate_up launch bytes = experts hit ({self.hit}) "
+                                  f"x (packed gate_up weights + scales + zero-points) + activations in/out")
+        return dict(bound="tensor", per_launch=ops, unit="TOPS", scale=1e12, peak=2.0 * peaks["bf16_sus"],
+                    kernel="gate_up",
+                    peak_note=f"2 x bf16_tflops_sustained ({peaks['source']}); gate_up launch ops = 2*pairs*H*2I")
+
+    def config(self):
+        return {"workload": (f"{self.name}: T={self.T} H={self.H} E={self.E} top-{self.topk} I={self.I} "
+                             f"{'symmetric' if self.sym else 'asymmetric+zero-point'} int4 g={self.group}"
+                             + (f", Zipf({self.zipf}) logits" if self.zipf else "")),
+                "T": self.T, "H": self.H, "E": self.E, "topk": self.topk, "I": self.I, "group": self.group,
+                "experts_hit": getattr(self, "hit", None),
+                "l2": f"expert weights {self.E * (3 * self.H * self.I) / 2 / 2**20:.0f} MiB vs L2 126 MiB"}
+
+    def e2e_setup(self):
+        import torch
+        self.X_pin = self.X_host.pin_memory()
+        self.L_pin = self.L_host.pin_memory()
+        self.out_pin = torch.empty(self.T, self.H, dtype=torch.bfloat16).pin_memory()
+        self.X2 = torch.empty_like(self.X)
+        self.L2 = torch.empty_like(self.L)
+        return self.X_pin.numel() * 2 + self.L_pin.numel() * 4, self.out_pin.numel() * 2
+
+    def e2e_step(self, i):
+        self.X2.copy_(self.X_pin, non_blocking=True)
+        self.L2.copy_(self.L_pin, non_blocking=True)
+        r = self.m.w4a8_moe_grouped_gemm(self.X2, self.L2, self.topk, self.w1, self.w2, workspace=self.ws,
+                                         out=self.out)
+        self.out_pin.copy_(r["out"], non_blocking=True)
+
+    def oracle_step_setup(self, n_tokens):
+        import numpy as np
+        import oracle as O
+        import torch
+        rng = np.random.default_rng(0)
+        toks = np.sort(rng.choice(self.T, n_tokens, replace=False))
+        Xb = self.X_host.view(torch.int16).numpy().view(np.uint16)[toks]
+        L = self.L_host.numpy()[toks]
+        idx, _, _ = O.route(L, self.topk)
+        need = sorted(set(int(e) for e in idx.ravel()))
+        codes1, codes2 = {}, {}
+        for e in need:  # weight quantization is offline: prepared here, untimed
+            codes1[e] = O.quant_weights(self._weight(e, 0, "cpu").numpy(), self.group, self.sym)[:3]
+            codes2[e] = O.quant_weights(self._weight(e, 1, "cpu").numpy(), self.group, self.sym)[:3]
+            if self.sym:
+                codes1[e] = (codes1[e][0], codes1[e][1], None)
+                codes2[e] = (codes2[e][0], codes2[e][1], None)
+        self._orc = (O, Xb, L, codes1, codes2)
+        return n_tokens / self.T
+
+    def oracle_step(self):
+        O, Xb, L, c1, c2 = self._orc
+        idx, p, _ = O.route(L, self.topk)
+        ex1 = [c1.get(e, (None, None, None)) for e in range(self.E)]
+        ex2 = [c2.get(e, (None, None, None)) for e in range(self.E)]
+        O.moe_forward(Xb, L, self.topk, ex1, ex2, self.group)
+
+
+def make_workload(name, M):
+    if name in ("decode", "prefill"):
+        return LinearWorkload(name, M if M else (32 if name == "decode" else 8192))
+    return MoEWorkload(name)
+
+
+# ------------------------------------------------------------- timing ---
+
+def capture(torch, fn, n, with_events=0):
+    """Captures n steps (fn(i, ev)) into one CUDA graph; with_events = number
+    of timing events per step handed to fn (recorded as graph nodes)."""
+    evs = [tuple(torch.cuda.Event(enable_timing=True, external=True) for _ in range(with_events))
+           for _ in range(n)] if with_events else [None] * n
+    for ev in evs:  # torch creates the CUDA event on its first record
+        for e in ev or ():
+            e.record()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fn(0, None)  # one eager call on the capture stream (library state, attributes)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=s):
+            for i in range(n):
+                fn(i, evs[i])
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    return g, evs
+
+
+def dist_setup(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier_sync(torch, world):
+    torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(torch, world, v):
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def run_ours(args, world, rank, local):
+    import torch
+    import moe_linear_layers_w4a8_b200 as m
+    m.load_library()  # fails loudly without the CUDA library
+    peaks = measured_peaks()
+    wl = make_workload(args.workload, args.m)
+    wl.setup()
+    K, W = args.steps, args.warmup
+    unit_scale, unit, meaning = wl.units()
+    roof = wl.kernel_roofline(peaks)
+
+    # graphs: warm-up graph (W steps), timed graph(s) of length Lg, the last
+    # replay with events around the dominant kernel.
+    Lg = max(1, min(K, 64 if args.workload in ("decode",) else 8))
+    reps, rem = divmod(K, Lg)
+    gw, _ = capture(torch, wl.step, max(W, 1))
+    gt, _ = capture(torch, wl.step, Lg)
+    gev, evs = capture(torch, wl.step, Lg, with_events=2 if isinstance(wl, LinearWorkload) else 8)
+    grem = capture(torch, wl.step, rem)[0] if rem else None
+
+    for _ in range(1 if W else 0):
+        gw.replay()
+    barrier_sync(torch, world)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    with sampler:
+        start.record()
+        for r in range(reps):
+            (gev if r == reps - 1 else gt).replay()
+        if grem is not None:
+            grem.replay()
+        end.record()
+        torch.cuda.synchronize()
+    barrier_sync(torch, world)
+    t_ms = start.elapsed_time(end)
+    t_ms = max_over_ranks(torch, world, t_ms)
+    ms_per_step = t_ms / K
+    value = unit_scale * K * world / (t_ms / 1e3)
+
+    # dominant-kernel time: events around its launches in the last replay
+    stage_ms = None
+    if reps > 0 and isinstance(wl, LinearWorkload):
+        k_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    elif reps > 0:
+        stage_ms = {name: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs)
+                    for i, name in enumerate(wl.STAGES)}
+        k_ms = stage_ms[roof["kernel"]]
+    else:
+        k_ms = ms_per_step
+    achieved = roof["per_launch"] / roof["scale"] / (k_ms / 1e3)
+    roofline = {"bound": roof["bound"], "achieved": round(achieved, 2), "peak": round(roof["peak"], 1),
+                "unit": roof["unit"], "frac": round(achieved / roof["peak"], 4),
+                "traffic": traffic_from_profiles(args.workload, roof), "kernel_ms": round(k_ms, 5),
+                "peak_source": roof["peak_note"], "algorithmic_per_launch": roof["per_launch"]}
+    if roof["bound"] == "hbm":
+        roofline["frac_note"] = "of measured" if peaks["source"] == "measured" else "of fallback"
+
+    # end to end through the public API with host buffers
+    del gw, gt, gev, grem
+    torch.cuda.synchronize()
+    h2d, d2h = wl.e2e_setup()
+    Ke = max(1, min(K, 2000 if args.workload == "decode" else max(10, K // 4)))
+    for i in range(min(W, 20)):
+        wl.e2e_step(i)
+    barrier_sync(torch, world)
+    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s2.record()
+    for i in range(Ke):
+        wl.e2e_step(i)
+    e2.record()
+    torch.cuda.synchronize()
+    te = max_over_ranks(torch, world, s2.elapsed_time(e2))
+    e2e_value = unit_scale * Ke * world / (te / 1e3)
+
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": unit, "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": round(ms_per_step, 6), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+        "config": dict(wl.config(), quantity=meaning, parallelism=f"replicas x{world}",
+                       global_batch=(getattr(wl, "M", None) or getattr(wl, "T", None)) * world),
+        "roofline": roofline,
+        "e2e": {"value": round(e2e_value, 3), "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": Ke},
+        "gpu_launches": wl.launches_per_step * K,
+        "clocks": sampler.summary(),
+    }
+    if stage_ms is not None:
+        roofline["stage_ms"] = {k: round(v, 5) for k, v in stage_ms.items()}
+        roofline["kernel"] = "w4a8_gemm_tc_kernel (gate_up)"
+    else:
+        roofline["kernel"] = "w4a8_gemm_tc_kernel"
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, unit_scale, unit)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def traffic_from_profiles(workload, roof):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary (profiles/*.json), or None when no current capture exists."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d.get(workload)
+    except Exception:
+        return None
+
+
+def cpu_baseline(wl, unit_scale, unit, budget_s=12.0):
+    """The oracle, as it stands, on a bounded sample of the same workload."""
+    import oracle as O
+    O.build()
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    frac, sample = _oracle_sample(wl)
+    t0 = time.perf_counter()
+    wl.oracle_step()
+    one = time.perf_counter() - t0
+    reps = max(1, min(50, int(budget_s / max(one, 1e-6))))
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        wl.oracle_step()
+    dt = (time.perf_counter() - t0) / reps
+    return {"value": round(unit_scale * frac / dt, 6), "unit": unit, "cores": cores, "kind": "oracle",
+            "sample": f"{sample}; {reps} repetitions, {dt * 1e3:.1f} ms each"}
+
+
+def _oracle_sample(wl):
+    if isinstance(wl, LinearWorkload):
+        n = wl.N if wl.decode else 256
+        frac = wl.oracle_step_setup(n) if wl.decode else _linear_row_sample(wl, 16)
+        return frac, (f"all {wl.N} output columns of the M={wl.M} decode step (weight quantization untimed)"
+                      if wl.decode else f"16 of {wl.M} rows x all {wl.N} columns")
+    n = min(wl.T, 8 if wl.T > 64 else 4)
+    return wl.oracle_step_setup(n), f"{n} of {wl.T} tokens through the whole layer"
+
+
+def _linear_row_sample(wl, rows):
+    import numpy as np
+    import oracle as O
+    import torch
+    W = wl._W_host()
+    codes, s, _, _ = O.quant_weights(W, wl.group, True)
+    Xb = wl.X_host.view(torch.int16).numpy().view(np.uint16)[:rows].copy()
+
+    def step():
+        O.linear(Xb, codes, s, None, wl.group)
+    wl.oracle_step = step
+    return rows / wl.M
+
+
+def run_reference(args, world, rank):
+    """Reference arm: the CPU oracle on the machine's host cores (rank 0 only)."""
+    if rank != 0:
+        return
+    import oracle as O
+    O.build()
+    wl = make_workload(args.workload, args.m)
+    # host-side copies of the inputs only (no GPU work on this arm)
+    if isinstance(wl, LinearWorkload):
+        from synth import gen_linear
+        inp = gen_linear(wl.M, wl.K, wl.N, seed=0, n_outliers=8, outlier_scale=50.0)
+        wl.X_host = inp.X
+        wl.w_bytes = wl.N * wl.K // 2 + (wl.K // wl.group) * wl.N * 4
+    else:
+        from synth import gen_moe_activations
+        inp = gen_moe_activations(wl.T, wl.H, wl.E, seed=0, zipf=wl.zipf)
+        wl.X_host, wl.L_host = inp.X, inp.logits
+    unit_scale, unit, meaning = wl.units()
+    K, W = args.steps, args.warmup
+    # size the per-step sample so that all K + W steps take about a minute
+    budget = 60.0
+    if isinstance(wl, LinearWorkload):
+        n_full = wl.N if wl.decode else wl.M
+        probe = max(64, n_full // 64)
+        if wl.decode:
+            wl.oracle_step_setup(probe)
+        else:
+            _linear_row_sample(wl, 1)
+        t0 = time.perf_counter(); wl.oracle_step(); t_probe = time.perf_counter() - t0
+        per_step = budget / (K + W)
+        n = int(max(1, min(n_full, probe * per_step / max(t_probe, 1e-9))))
+        if wl.decode:
+            frac = wl.oracle_step_setup(max(64, n) if n >= 64 else max(1, n))
+            sample = f"{max(64, n) if n >= 64 else max(1, n)} of {wl.N} output columns, all {wl.M} rows"
+        else:
+            frac = _linear_row_sample(wl, max(1, min(n, 64)))
+            sample = f"{max(1, min(n, 64))} of {wl.M} rows x all {wl.N} columns"
+    else:
+        frac = wl.oracle_step_setup(1)
+        sample = f"1 of {wl.T} tokens through the whole layer"
+    for _ in range(W):
+        wl.oracle_step()
+    t0 = time.perf_counter()
+    for _ in range(K):
+        wl.oracle_step()
+    dt = time.perf_counter() - t0
+    value = unit_scale * frac * K / dt
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": unit, "n_gpus": world, "steps": K,
+        "warmup": W, "ms_per_step": round(dt / K * 1e3, 6), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+        "config": dict(wl.config(), quantity=meaning),
+        "cpu_baseline": {"value": round(value, 6), "unit": unit, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="decode",
+                    choices=["decode", "prefill", "moe_sym", "moe_asym_decode", "moe_asym_prefill"])
+    ap.add_argument("--m", type=int, default=None, help="rows of the linear workloads")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.steps is None:
+        args.steps = DEFAULT_STEPS[args.workload]
+    args.warmup = max(args.warmup, 3)
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, world, rank)
+        return
+    world, rank, local = dist_setup(args)
+    run_ours(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

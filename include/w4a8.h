@@ -229,6 +229,20 @@ W4A8_API w4a8_status w4a8_moe_grouped_gemm(const uint16_t* X, const float* logit
                                   void* workspace, size_t ws_bytes,
                                   int32_t* dev_status, void* stream);
 
+/* w4a8_moe_grouped_gemm_profiled — the same call, which also records the
+ * caller's CUDA events (cudaEvent_t passed as void*; NULL entries skipped)
+ * on `stream` at its stage boundaries, for timing: stage_events[0] before
+ * routing, [1] before dispatch, [2] before quantizing X, [3] before gate_up,
+ * [4] before quantizing h, [5] before down, [6] before the combine, [7] after
+ * it.  Events are recorded as external events, so they also work inside a
+ * stream capture.  stage_events may be NULL. */
+W4A8_API w4a8_status w4a8_moe_grouped_gemm_profiled(
+    const uint16_t* X, const float* logits, int T, int E, int topk,
+    const uint8_t* w1_packed, const float* w1_s, const uint8_t* w1_z, const w4a8_wdesc* w1,
+    const uint8_t* w2_packed, const float* w2_s, const uint8_t* w2_z, const w4a8_wdesc* w2,
+    uint16_t* out, int32_t* topk_idx_out, float* topk_w_out, int32_t* expert_offsets_out,
+    void* workspace, size_t ws_bytes, int32_t* dev_status, void* stream, void* const* stage_events);
+
 /* Byte offsets of the MoE intermediates inside the workspace, for stage-wise
  * inspection (tests): perm int32 [T*k] (position -> t*k+j), inv int32 [T*k],
  * qx int8 [T*k][H] and sx fp32 [T*k] in dispatch order, h bf16 [T*k][I],

@@ -113,6 +113,8 @@ def load_library():
         L.w4a8_moe_grouped_gemm.restype = st
         L.w4a8_moe_grouped_gemm.argtypes = [P, P, I, I, I, P, P, P, ctypes.POINTER(WDesc), P, P, P,
                                             ctypes.POINTER(WDesc), P, P, P, P, P, S, P, P]
+        L.w4a8_moe_grouped_gemm_profiled.restype = st
+        L.w4a8_moe_grouped_gemm_profiled.argtypes = L.w4a8_moe_grouped_gemm.argtypes + [P]
         L.w4a8_get_device_status.restype = st
         L.w4a8_get_device_status.argtypes = [P, P]
         L.w4a8_selftest_bounded_wait.restype = st
@@ -202,15 +204,16 @@ def w4a8_pack_expert_weights(make_weight, E: int, K: int, N: int, group: int, sy
 
 # ------------------------------------------------------------- activation --
 
-def w4a8_quant_act(X: torch.Tensor, group_for_rowsum: int = 0, status: Optional[torch.Tensor] = None):
+def w4a8_quant_act(X: torch.Tensor, group_for_rowsum: int = 0, status: Optional[torch.Tensor] = None,
+                   q_out: Optional[torch.Tensor] = None, s_out: Optional[torch.Tensor] = None):
     """Per-token INT8 quantization of X bf16 [M, K] -> (q int8, s_x fp32, rowsum|None)."""
     L = load_library()
     _need_cuda(X)
     if X.dtype != torch.bfloat16 or X.dim() != 2 or X.stride(1) != 1:
         raise W4A8Error(1, "X must be bf16 [M, K] with unit column stride")
     M, K = X.shape
-    q = torch.empty(M, K, dtype=torch.int8, device=X.device)
-    s = torch.empty(M, dtype=torch.float32, device=X.device)
+    q = q_out if q_out is not None else torch.empty(M, K, dtype=torch.int8, device=X.device)
+    s = s_out if s_out is not None else torch.empty(M, dtype=torch.float32, device=X.device)
     rs = (torch.empty(M, K // group_for_rowsum, dtype=torch.int32, device=X.device)
           if group_for_rowsum else None)
     code = L.w4a8_quant_act(_p(X), M, K, X.stride(0), int(group_for_rowsum), _p(q), _p(s), _p(rs),
@@ -263,9 +266,10 @@ def w4a8_gemm_debug_partials(qx, s_x, w: PackedWeight, out=None, workspace=None,
     return Y, P
 
 
-def w4a8_linear(X: torch.Tensor, w: PackedWeight, out=None, workspace=None, status=None) -> torch.Tensor:
+def w4a8_linear(X: torch.Tensor, w: PackedWeight, out=None, workspace=None, status=None,
+                q_buf=None, s_buf=None) -> torch.Tensor:
     """Per-token quantization of X followed by the W4A8 GEMM."""
-    q, s, _ = w4a8_quant_act(X, status=status)
+    q, s, _ = w4a8_quant_act(X, status=status, q_out=q_buf, s_out=s_buf)
     return w4a8_gemm(q, s, w, out=out, workspace=workspace, status=status)
 
 
@@ -286,9 +290,12 @@ def w4a8_moe_workspace_layout(T: int, E: int, topk: int, w1: PackedWeight, w2: P
 
 def w4a8_moe_grouped_gemm(X: torch.Tensor, logits: torch.Tensor, topk: int, w1: PackedWeight,
                           w2: PackedWeight, workspace: Optional[torch.Tensor] = None,
-                          status: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None):
+                          status: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                          stage_events=None):
     """One MoE expert layer (route, dispatch, gate_up + SiLU*up, down, combine).
-    Returns dict(out, topk_idx, topk_w, expert_offsets, workspace)."""
+    Returns dict(out, topk_idx, topk_w, expert_offsets, workspace).
+    stage_events: optional list of 8 torch.cuda.Event recorded at the stage
+    boundaries (see w4a8_moe_grouped_gemm_profiled)."""
     L = load_library()
     _need_cuda(X, logits)
     if X.dtype != torch.bfloat16 or logits.dtype != torch.float32:
@@ -308,12 +315,16 @@ def w4a8_moe_grouped_gemm(X: torch.Tensor, logits: torch.Tensor, topk: int, w1: 
     idx = torch.empty(T, topk, dtype=torch.int32, device=dev)
     pw = torch.empty(T, topk, dtype=torch.float32, device=dev)
     offs = torch.empty(E + 1, dtype=torch.int32, device=dev)
-    code = L.w4a8_moe_grouped_gemm(
-        _p(X), _p(logits), T, E, int(topk),
-        _p(w1.packed), _p(w1.s_w), _p(w1.z), ctypes.byref(w1.desc),
-        _p(w2.packed), _p(w2.s_w), _p(w2.z), ctypes.byref(w2.desc),
-        _p(out), _p(idx), _p(pw), _p(offs), _p(workspace),
-        workspace.numel() * workspace.element_size(), _p(status), _stream(dev))
+    args = [_p(X), _p(logits), T, E, int(topk),
+            _p(w1.packed), _p(w1.s_w), _p(w1.z), ctypes.byref(w1.desc),
+            _p(w2.packed), _p(w2.s_w), _p(w2.z), ctypes.byref(w2.desc),
+            _p(out), _p(idx), _p(pw), _p(offs), _p(workspace),
+            workspace.numel() * workspace.element_size(), _p(status), _stream(dev)]
+    if stage_events is None:
+        code = L.w4a8_moe_grouped_gemm(*args)
+    else:
+        evs = (ctypes.c_void_p * 8)(*[None if e is None else ctypes.c_void_p(e.cuda_event) for e in stage_events])
+        code = L.w4a8_moe_grouped_gemm_profiled(*args, evs)
     _check(code, "w4a8_moe_grouped_gemm")
     return dict(out=out, topk_idx=idx, topk_w=pw, expert_offsets=offs, workspace=workspace)
 

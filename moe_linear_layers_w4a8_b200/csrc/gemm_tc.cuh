@@ -11,26 +11,29 @@
 //
 // Design (B200):
 //   * Swap-AB: the 128 MMA rows (M) are weight output columns n, the MMA N
-//     dimension (BN = 16..128) is tokens.  A 128 x 128 x 128 int8 MMA block
-//     then needs only 16 KB of unpacked weights, each epilogue thread owns
-//     one weight column (so s_w[g,n] is a per-thread scalar), and decode-size
-//     M runs on the same kernel with BN = 16.
-//   * Warp roles (448 threads): warp 0 issues TMA / bulk copies; warp 1
-//     allocates TMEM and one lane issues tcgen05.mma; warps 2-5 unpack the
-//     4-bit codes (minus the zero-point) into the swizzled int8 A tile;
-//     warps 6-13 drain TMEM per group and accumulate in fp32 registers.
-//   * TMEM holds two int32 partial buffers (double-buffered across groups).
-//     Each buffer is pre-filled with 0x4B400000 before a group's MMAs, so
-//     after them it holds the bits of the float 12582912 + P (|P| < 2^22):
-//     one FADD turns it into P exactly, one FFMA applies s_w.
-//   * K is walked one quantization group per pipeline stage (64 or 128
-//     bytes of K per row = one 64B / 128B swizzle atom row).
+//     dimension (BN = 16..128) is tokens.  Each epilogue thread owns one
+//     weight column (so s_w[g,n] is a per-thread scalar), and decode-size M
+//     runs on the same kernel with BN = 16.
+//   * The unpacked int8 weight tile lives in TMEM (tcgen05.mma with A from
+//     TMEM): each unpack thread turns one row of packed codes into int8 in
+//     registers and writes the whole row of the group with one tcgen05.st,
+//     so the only shared-memory traffic per step is the packed codes and the
+//     activation tile.
+//   * Warp roles (512 threads): warps 0-3 unpack (warp q owns TMEM lanes /
+//     weight rows 32q..32q+31), warps 4-11 drain the partial sums, warp 12
+//     brings packed codes (TMA bulk copies, deep ring), warp 13 brings
+//     activation tiles (tiled TMA), one lane of warp 14 issues the MMAs.
+//   * TMEM holds NACC int32 partial buffers.  Each is pre-filled with
+//     0x4B400000 before a group's MMAs, so afterwards it holds the bits of
+//     the float 12582912 + P (|P| < 2^22): one FADD turns it into P exactly,
+//     one FFMA applies s_w.
+//   * K is walked one quantization group per pipeline step.
 //   * Persistent: each CTA owns a contiguous range of (tile, group) units.
 //     Ranges that split a tile (split-K) write fp32 partial tiles that a
 //     second kernel sums in a fixed order.
-//   * Every mbarrier wait is bounded (globaltimer); on expiry the CTA
-//     records W4A8_ERR_TIMEOUT, drains its in-flight copies and MMAs, frees
-//     TMEM and exits.
+//   * Every mbarrier wait is bounded; on expiry the CTA records
+//     W4A8_ERR_TIMEOUT, drains its in-flight copies and MMAs, frees TMEM and
+//     exits.
 #pragma once
 
 #include <cstdint>
@@ -70,35 +73,45 @@ struct GemmParams {
     unsigned long long wait_ns;
 };
 
-constexpr int kGemmThreads = 448;
+constexpr int kGemmThreads = 512;  // 4 unpack, 8 epilogue, 2 producer, 1 MMA, 1 spare warp
 constexpr int kNumEpiWarps = 8;
 constexpr uint32_t kMagicBits = 0x4B400000u;  // float 12582912 = 1.5 * 2^23
 constexpr float kMagicF = 12582912.0f;
 
-template <int BN, int GROUP, int S, int SA>
+template <int BN, int GROUP, int SP, int SA, int NACC_>
 struct GemmCfg {
-    static constexpr int A_STAGE = 128 * GROUP;
+    // P ring: packed codes + zero-points (TMA -> unpack warps).
+    // A ring: activation tile (TMA, shared memory) + unpacked weight tile
+    //         (unpack warps, TMEM), both drained by the MMA.
+    static constexpr int NACC = NACC_;           // TMEM partial buffers
+    static constexpr int GW = GROUP / 4;         // TMEM columns of one unpacked group
+    static constexpr int A_COL0 = NACC * BN;     // first TMEM column of the A ring
     static constexpr int ACT_STAGE = BN * GROUP;
-    static constexpr int PK_HALF = 32 * GROUP;  // one 64-column block of one group
+    static constexpr int PK_HALF = 32 * GROUP;   // one 64-column block of one group
     static constexpr int PK_STAGE = 2 * PK_HALF;
     static constexpr int Z_STAGE = 128;
     static constexpr int XBUF = 64 * BN * 4;
-    static constexpr int OFF_A = 0;
-    static constexpr int OFF_ACT = OFF_A + SA * A_STAGE;
-    static constexpr int OFF_PK = OFF_ACT + S * ACT_STAGE;
-    static constexpr int OFF_Z = OFF_PK + S * PK_STAGE;
-    static constexpr int OFF_X = OFF_Z + S * Z_STAGE;
+    static constexpr int SWS = 32;               // s_w ring (128 fp32 per step)
+    static constexpr int OFF_ACT = 0;
+    static constexpr int OFF_PK = OFF_ACT + SA * ACT_STAGE;
+    static constexpr int OFF_Z = OFF_PK + SP * PK_STAGE;
+    static constexpr int OFF_SW = OFF_Z + SP * Z_STAGE;
+    static constexpr int OFF_X = OFF_SW + SWS * 512;
     static constexpr int OFF_BAR = OFF_X + XBUF;
-    static constexpr int NUM_BARS = 2 * S + 2 * SA + 4 + 1;
+    static constexpr int NUM_BARS = 2 * SP + 3 * SA + 2 * NACC + 2 * SWS + 1;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
     static constexpr int BYTES = OFF_MISC + 16;
-    static constexpr int SMEM = BYTES + 1024;  // slack for 1024-byte alignment
-    static constexpr int CH = BN / 2;          // accumulator columns per epilogue thread
-    static constexpr uint32_t TMEM_COLS = (2 * BN < 32) ? 32 : 2 * BN;
+    static constexpr int SMEM = BYTES + 1024;    // slack for 1024-byte alignment
+    static constexpr int CH = BN / 2;            // accumulator columns per epilogue thread
+    static constexpr int TMEM_USED = A_COL0 + SA * GW;
+    static constexpr uint32_t TMEM_COLS = TMEM_USED <= 32 ? 32 : TMEM_USED <= 64 ? 64 : TMEM_USED <= 128 ? 128
+                                          : TMEM_USED <= 256 ? 256 : 512;
     static constexpr uint32_t IDESC = idesc_i8(BN);
     static_assert(BN == 16 || BN == 32 || BN == 64 || BN == 128, "BN");
     static_assert(GROUP == 64 || GROUP == 128, "GROUP");
-    static_assert(A_STAGE % 1024 == 0 && ACT_STAGE % 1024 == 0, "swizzle atoms need 1024-byte stages");
+    static_assert(ACT_STAGE % 1024 == 0, "swizzle atoms need 1024-byte stages");
+    static_assert(SA >= 2 && SP >= 2 && NACC >= 2, "rings");
+    static_assert(TMEM_USED <= 512, "TMEM columns");
     static_assert(SMEM <= 227 * 1024, "shared memory");
 };
 
@@ -172,25 +185,32 @@ __device__ __forceinline__ void cta_units(const GemmParams& p, long long& u0, lo
     if (u0 > U) u0 = U;
 }
 
-template <int BN, int GROUP, int S, int SA>
+constexpr int kUnpackWarps = 4;
+
+constexpr int kWarpPack = 12, kWarpAct = 13, kWarpMma = 14;
+
+template <int BN, int GROUP, int SP, int SA, int NACC>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     w4a8_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act, const GemmParams p) {
-    using C = GemmCfg<BN, GROUP, S, SA>;
+    using C = GemmCfg<BN, GROUP, SP, SA, NACC>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* sA = smem + C::OFF_A;
     uint8_t* sAct = smem + C::OFF_ACT;
     uint8_t* sPk = smem + C::OFF_PK;
     uint8_t* sZ = smem + C::OFF_Z;
+    float* sSW = reinterpret_cast<float*>(smem + C::OFF_SW);
     float* sX = reinterpret_cast<float*>(smem + C::OFF_X);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-    uint64_t* full = bars;                 // [S]  TMA landed (packed + z + act)
-    uint64_t* empty = bars + S;            // [S]  unpack warps + MMA done with stage
-    uint64_t* a_full = bars + 2 * S;       // [SA] A tile unpacked
-    uint64_t* a_empty = a_full + SA;       // [SA] MMA done with A tile
-    uint64_t* acc_full = a_empty + SA;     // [2]  partial buffer ready
-    uint64_t* acc_empty = acc_full + 2;    // [2]  partial buffer drained + re-filled
-    uint64_t* drain = acc_empty + 2;       // [1]
+    uint64_t* p_full = bars;                 // [SP] packed codes (+ z) landed
+    uint64_t* p_empty = p_full + SP;         // [SP] the 4 unpack warps read them
+    uint64_t* act_full = p_empty + SP;       // [SA] activation tile landed
+    uint64_t* a_full = act_full + SA;        // [SA] weight tile unpacked into TMEM
+    uint64_t* a_empty = a_full + SA;         // [SA] MMA done with both
+    uint64_t* acc_full = a_empty + SA;       // [NACC] partial buffer ready
+    uint64_t* acc_empty = acc_full + NACC;   // [NACC] partial buffer drained + re-armed
+    uint64_t* sw_full = acc_empty + NACC;    // [SWS] group scales of the step landed
+    uint64_t* sw_empty = sw_full + C::SWS;   // [SWS] the 8 epilogue warps read them
+    uint64_t* drain = sw_empty + C::SWS;     // [1]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
     int* abort_flag = reinterpret_cast<int*>(smem + C::OFF_MISC + 4);
 
@@ -198,17 +218,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < S; ++i) {
-            mbar_init(&full[i], 1);
-            mbar_init(&empty[i], 4 + 1);
+        for (int i = 0; i < SP; ++i) {
+            mbar_init(&p_full[i], 1);
+            mbar_init(&p_empty[i], kUnpackWarps);
         }
         for (int i = 0; i < SA; ++i) {
-            mbar_init(&a_full[i], 4);
+            mbar_init(&act_full[i], 1);
+            mbar_init(&a_full[i], kUnpackWarps);
             mbar_init(&a_empty[i], 1);
         }
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < NACC; ++i) {
             mbar_init(&acc_full[i], 1);
             mbar_init(&acc_empty[i], kNumEpiWarps);
+        }
+        for (int i = 0; i < C::SWS; ++i) {
+            mbar_init(&sw_full[i], 1);
+            mbar_init(&sw_empty[i], kNumEpiWarps);
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -216,7 +241,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         fence_proxy_async_smem();
         prefetch_tmap(&tmap_act);
     }
-    if (warp == 1) {
+    if (warp == kWarpMma) {
         tmem_alloc(tmem_slot, C::TMEM_COLS);
         tmem_relinquish();
     }
@@ -224,177 +249,186 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    const WaitCtx wc{abort_flag, p.status, p.wait_ns};
+    const WaitCtx wc{abort_flag, p.status, wait_cycles_for_ns(p.wait_ns)};
 
     long long u0, u1, Q;
     cta_units(p, u0, u1, Q);
     const int G = p.G;
+    const long long nsteps = u1 - u0;  // one step = one K-group of one tile
 
-    if (warp == 0) {
-        // ------------------------------------------------------ producer --
+    if (warp == kWarpPack || warp == kWarpAct) {
+        // ------------------------------------------------------ producers --
         if (lane == 0) {
-            Ring st;
+            const bool pack = warp == kWarpPack;
+            const int ring = pack ? SP : SA;
             long long issued = 0;
             bool ok = true;
-            for (long long u = u0; u < u1 && ok;) {
-                const long long t = u / G;
-                const int gb = (int)(u % G);
-                const int ge = (int)min((long long)G, gb + (u1 - u));
-                const TileInfo ti = decode_tile<BN>(p, t);
-                int nb0, nb1;
-                tile_blocks(p, ti.nt, nb0, nb1);
-                const uint8_t* wbase = p.packed + (long long)ti.e * p.packed_estride;
-                const uint8_t* zrow_base = p.symmetric ? nullptr : p.z + (long long)ti.e * p.sw_estride;
-                for (int gi = gb; gi < ge; ++gi) {
-                    if (!wait_bounded(&empty[st.idx], st.phase ^ 1u, wc)) { ok = false; break; }
-                    uint32_t bytes = C::PK_HALF + C::ACT_STAGE;
+            long long t = u0 / G;
+            int gi = (int)(u0 % G);
+            long long cur_t = -1;
+            TileInfo ti{};
+            int nb0 = 0, nb1 = -1;
+            Ring rs, rw;  // this producer's ring; s_w ring (activation producer)
+            for (long long i = 0; i < nsteps; ++i) {
+                if (t != cur_t) {
+                    ti = decode_tile<BN>(p, t);
+                    tile_blocks(p, ti.nt, nb0, nb1);
+                    cur_t = t;
+                }
+                const uint32_t s = rs.idx;
+                if (pack) {
+                    if (!wait_bounded(&p_empty[s], rs.phase ^ 1u, wc)) { ok = false; break; }
+                    uint32_t bytes = C::PK_HALF;
                     if (nb1 >= 0) bytes += C::PK_HALF;
                     if (!p.symmetric) bytes += (nb1 >= 0) ? 128 : 64;
-                    mbar_arrive_expect_tx(&full[st.idx], bytes);
-                    uint8_t* pk = sPk + st.idx * C::PK_STAGE;
-                    bulk_load(pk, wbase + ((long long)nb0 * G + gi) * C::PK_HALF, C::PK_HALF, &full[st.idx]);
+                    mbar_arrive_expect_tx(&p_full[s], bytes);
+                    const uint8_t* wbase = p.packed + (long long)ti.e * p.packed_estride;
+                    uint8_t* pk = sPk + s * C::PK_STAGE;
+                    bulk_load(pk, wbase + ((long long)nb0 * G + gi) * C::PK_HALF, C::PK_HALF, &p_full[s]);
                     if (nb1 >= 0)
                         bulk_load(pk + C::PK_HALF, wbase + ((long long)nb1 * G + gi) * C::PK_HALF, C::PK_HALF,
-                                  &full[st.idx]);
+                                  &p_full[s]);
                     if (!p.symmetric) {
-                        const uint8_t* zr = zrow_base + (long long)gi * p.N;
-                        bulk_load(sZ + st.idx * C::Z_STAGE, zr + 64 * nb0, 64, &full[st.idx]);
-                        if (nb1 >= 0) bulk_load(sZ + st.idx * C::Z_STAGE + 64, zr + 64 * nb1, 64, &full[st.idx]);
+                        const uint8_t* zr = p.z + (long long)ti.e * p.sw_estride + (long long)gi * p.N;
+                        bulk_load(sZ + s * C::Z_STAGE, zr + 64 * nb0, 64, &p_full[s]);
+                        if (nb1 >= 0) bulk_load(sZ + s * C::Z_STAGE + 64, zr + 64 * nb1, 64, &p_full[s]);
                     }
-                    tma_load_2d(sAct + st.idx * C::ACT_STAGE, &tmap_act, &full[st.idx], gi * GROUP, ti.row0);
-                    ++issued;
-                    st.next(S);
+                } else {
+                    // group scales of the step's 128 weight rows (read by the epilogue)
+                    const uint32_t w = rw.idx;
+                    if (!wait_bounded(&sw_empty[w], rw.phase ^ 1u, wc)) { ok = false; break; }
+                    mbar_arrive_expect_tx(&sw_full[w], (nb1 >= 0) ? 512 : 256);
+                    const float* swr = p.s_w + (long long)ti.e * p.sw_estride + (long long)gi * p.N;
+                    bulk_load(sSW + w * 128, swr + 64 * nb0, 256, &sw_full[w]);
+                    if (nb1 >= 0) bulk_load(sSW + w * 128 + 64, swr + 64 * nb1, 256, &sw_full[w]);
+                    rw.next(C::SWS);
+                    // activation tile
+                    if (!wait_bounded(&a_empty[s], rs.phase ^ 1u, wc)) { ok = false; break; }
+                    mbar_arrive_expect_tx(&act_full[s], C::ACT_STAGE);
+                    tma_load_2d(sAct + s * C::ACT_STAGE, &tmap_act, &act_full[s], gi * GROUP, ti.row0);
                 }
-                u += ge - gb;
+                rs.next(ring);
+                ++issued;
+                if (++gi == G) { gi = 0; ++t; }
             }
+            (void)ok;
             // Drain: wait for the last issue of every stage, so no copy is in
-            // flight into this CTA's shared memory when it exits.
-            Ring d = st;
-            const long long n_drain = issued < S ? issued : S;
-            for (long long i = 0; i < n_drain; ++i) {
-                // step back one stage
-                if (d.idx == 0) { d.idx = S - 1; d.phase ^= 1u; } else { --d.idx; }
-                WaitCtx wd{abort_flag, p.status, p.wait_ns};
-                volatile int no_abort = 0;
-                wd.abort = &no_abort;  // drain even after an abort
-                (void)wait_bounded(&full[d.idx], d.phase, wd);
+            // flight into shared memory when the CTA exits.
+            WaitCtx wd{abort_flag, p.status, wait_cycles_for_ns(p.wait_ns)};
+            volatile int no_abort = 0;
+            wd.abort = &no_abort;  // drain even after an abort
+            uint64_t* fullb = pack ? p_full : act_full;
+            Ring d = rs;
+            for (long long k = 0; k < issued && k < ring; ++k) {
+                if (d.idx == 0) { d.idx = ring - 1; d.phase ^= 1u; } else { --d.idx; }
+                (void)wait_bounded(&fullb[d.idx], d.phase, wd);
+            }
+            if (!pack) {
+                const long long nsw = issued + (ok ? 0 : 1);  // an s_w copy may precede a failed wait
+                Ring dw = rw;
+                for (long long k = 0; k < nsw && k < C::SWS; ++k) {
+                    if (dw.idx == 0) { dw.idx = C::SWS - 1; dw.phase ^= 1u; } else { --dw.idx; }
+                    (void)wait_bounded(&sw_full[dw.idx], dw.phase, wd);
+                }
             }
         }
-    } else if (warp == 1) {
+    } else if (warp == kWarpMma) {
         // ----------------------------------------------------- MMA issue --
         if (lane == 0) {
-            Ring st, sa, ac;
-            bool ok = true;
-            const uint32_t a_base = smem_u32(sA);
             const uint32_t b_base = smem_u32(sAct);
-            for (long long u = u0; u < u1 && ok;) {
-                const int gb = (int)(u % G);
-                const int ge = (int)min((long long)G, gb + (u1 - u));
-                for (int gi = gb; gi < ge; ++gi) {
-                    if (!wait_bounded(&full[st.idx], st.phase, wc)) { ok = false; break; }
-                    if (!wait_bounded(&a_full[sa.idx], sa.phase, wc)) { ok = false; break; }
-                    if (!wait_bounded(&acc_empty[ac.idx], ac.phase, wc)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint64_t adesc = umma_desc_kmajor(a_base + sa.idx * C::A_STAGE, GROUP);
-                    const uint64_t bdesc = umma_desc_kmajor(b_base + st.idx * C::ACT_STAGE, GROUP);
-                    const uint32_t d_tmem = tmem_base + ac.idx * BN;
+            Ring ra, rc;
+            for (long long i = 0; i < nsteps; ++i, ra.next(SA), rc.next(NACC)) {
+                const uint32_t sa = ra.idx;
+                const uint32_t ab = rc.idx;
+                if (!wait_bounded(&act_full[sa], ra.phase, wc)) break;
+                if (!wait_bounded(&a_full[sa], ra.phase, wc)) break;
+                if (!wait_bounded(&acc_empty[ab], rc.phase, wc)) break;
+                tc_fence_after();
+                const uint64_t bdesc = umma_desc_kmajor(b_base + sa * C::ACT_STAGE, GROUP);
+                const uint32_t a_tmem = tmem_base + C::A_COL0 + sa * C::GW;
+                const uint32_t d_tmem = tmem_base + ab * BN;
 #pragma unroll
-                    for (int kk = 0; kk < GROUP / 32; ++kk)
-                        mma_i8(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, C::IDESC, 1u);
-                    tc_commit(&empty[st.idx]);
-                    tc_commit(&a_empty[sa.idx]);
-                    tc_commit(&acc_full[ac.idx]);
-                    st.next(S);
-                    sa.next(SA);
-                    ac.next(2);
-                }
-                u += ge - gb;
+                for (int kk = 0; kk < GROUP / 32; ++kk)
+                    mma_i8_tmem_a(d_tmem, a_tmem + 8 * kk, bdesc + 2 * kk, C::IDESC, 1u);
+                tc_commit(&a_empty[sa]);
+                tc_commit(&acc_full[ab]);
             }
             // Drain: every MMA issued above completes before TMEM is freed.
             tc_commit(drain);
-            WaitCtx wd{abort_flag, p.status, p.wait_ns};
+            WaitCtx wd{abort_flag, p.status, wait_cycles_for_ns(p.wait_ns)};
             volatile int no_abort = 0;
             wd.abort = &no_abort;
             (void)wait_bounded(drain, 0, wd);
         }
-    } else if (warp < 6) {
+    } else if (warp < kUnpackWarps) {
         // ---------------------------------------------------------- unpack --
-        const int r = threadIdx.x - 64;  // A row 0..127
+        // Warp q turns rows 32q..32q+31 of every step's weight tile into int8
+        // and stores them in TMEM lanes 32q..32q+31 (row = lane).
+        const int r = warp * 32 + lane;
         const int half = r >> 6, rr = r & 63;
-        Ring st, sa;
-        bool ok = true;
-        for (long long u = u0; u < u1 && ok;) {
-            const long long t = u / G;
-            const int gb = (int)(u % G);
-            const int ge = (int)min((long long)G, gb + (u1 - u));
-            const TileInfo ti = decode_tile<BN>(p, t);
-            int nb0, nb1;
-            tile_blocks(p, ti.nt, nb0, nb1);
-            const bool row_valid = (half == 0) || (nb1 >= 0);
-            // Each byte: 0x80 | code (sym: code ^ 8 = q + 8), minus z (sym: 8),
-            // then ^ 0x80: the two's complement int8 of (q - z) in [-15, 15].
-            const uint32_t k1 = p.symmetric ? 0x88888888u : 0x80808080u;
-            for (int gi = gb; gi < ge; ++gi) {
-                if (!warp_wait_bounded(&full[st.idx], st.phase, wc)) { ok = false; break; }
-                uint4 w[GROUP / 32];
-                uint32_t zz = 0x08080808u;
-                if (row_valid) {
-                    const uint8_t* pk = sPk + st.idx * C::PK_STAGE + half * C::PK_HALF;
-#pragma unroll
-                    for (int c = 0; c < GROUP / 32; ++c)
-                        w[c] = *reinterpret_cast<const uint4*>(pk + (c * 64 + rr) * 16);
-                    if (!p.symmetric) zz = 0x01010101u * (uint32_t)sZ[st.idx * C::Z_STAGE + half * 64 + rr];
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[st.idx]);
-                if (!warp_wait_bounded(&a_empty[sa.idx], sa.phase ^ 1u, wc)) { ok = false; break; }
-                uint8_t* arow = sA + sa.idx * C::A_STAGE + r * GROUP;
-#pragma unroll
-                for (int c = 0; c < GROUP / 32; ++c) {
-                    uint4 lo4 = make_uint4(0, 0, 0, 0), hi4 = make_uint4(0, 0, 0, 0);
-                    if (row_valid) {
-                        const uint32_t ws[4] = {w[c].x, w[c].y, w[c].z, w[c].w};
-                        uint32_t lo[4], hi[4];
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            lo[i] = (((ws[i] & 0x0F0F0F0Fu) ^ k1) - zz) ^ 0x80808080u;
-                            hi[i] = ((((ws[i] >> 4) & 0x0F0F0F0Fu) ^ k1) - zz) ^ 0x80808080u;
-                        }
-                        lo4 = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-                        hi4 = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                    }
-                    // logical 16-byte chunks 2c (k = 32c..32c+15) and 2c+1
-                    int p0, p1;
-                    if (GROUP == 128) {
-                        p0 = (2 * c) ^ (r & 7);
-                        p1 = (2 * c + 1) ^ (r & 7);
-                    } else {
-                        p0 = (2 * c) ^ ((r >> 1) & 3);
-                        p1 = (2 * c + 1) ^ ((r >> 1) & 3);
-                    }
-                    *reinterpret_cast<uint4*>(arow + p0 * 16) = lo4;
-                    *reinterpret_cast<uint4*>(arow + p1 * 16) = hi4;
-                }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&a_full[sa.idx]);
-                st.next(S);
-                sa.next(SA);
+        const uint32_t lane_addr = ((uint32_t)(warp * 32)) << 16;
+        // Each byte: 0x80 | code (sym: code ^ 8 = q + 8), minus z (sym: 8),
+        // then ^ 0x80: the two's complement int8 of (q - z) in [-15, 15].
+        const uint32_t k1 = p.symmetric ? 0x88888888u : 0x80808080u;
+        long long cur_t = -1;
+        int nb1 = -1;
+        long long t = u0 / G;
+        int gi = (int)(u0 % G);
+        Ring rp, ra;
+        for (long long i = 0; i < nsteps; ++i, rp.next(SP), ra.next(SA)) {
+            if (t != cur_t) {
+                const TileInfo ti = decode_tile<BN>(p, t);
+                int nb0;
+                tile_blocks(p, ti.nt, nb0, nb1);
+                cur_t = t;
             }
-            u += ge - gb;
+            if (++gi == G) { gi = 0; ++t; }
+            const bool row_valid = (half == 0) || (nb1 >= 0);
+            const uint32_t ps = rp.idx;
+            if (!warp_wait_bounded(&p_full[ps], rp.phase, wc)) break;
+            uint4 w[GROUP / 32];
+            uint32_t zz = 0x08080808u;
+            const uint8_t* pk = sPk + ps * C::PK_STAGE + half * C::PK_HALF;
+#pragma unroll
+            for (int c = 0; c < GROUP / 32; ++c)
+                w[c] = row_valid ? *reinterpret_cast<const uint4*>(pk + (c * 64 + rr) * 16) : make_uint4(0, 0, 0, 0);
+            if (!p.symmetric) zz = 0x01010101u * (uint32_t)sZ[ps * C::Z_STAGE + r];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&p_empty[ps]);
+            // TMEM column 8c + j holds k = 32c + 4j .. 32c + 4j + 3
+            uint32_t out[C::GW];
+#pragma unroll
+            for (int c = 0; c < GROUP / 32; ++c) {
+                const uint32_t ws[4] = {w[c].x, w[c].y, w[c].z, w[c].w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint32_t lo = (((ws[j] & 0x0F0F0F0Fu) ^ k1) - zz) ^ 0x80808080u;
+                    const uint32_t hi = ((((ws[j] >> 4) & 0x0F0F0F0Fu) ^ k1) - zz) ^ 0x80808080u;
+                    out[8 * c + j] = row_valid ? lo : 0u;
+                    out[8 * c + 4 + j] = row_valid ? hi : 0u;
+                }
+            }
+            const uint32_t sa = ra.idx;
+            if (!warp_wait_bounded(&a_empty[sa], ra.phase ^ 1u, wc)) break;
+            tc_fence_after();
+            tmem_st32<C::GW>(tmem_base + lane_addr + C::A_COL0 + sa * C::GW, out);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&a_full[sa]);
         }
-    } else {
+    } else if (warp < kUnpackWarps + kNumEpiWarps) {
         // -------------------------------------------------------- epilogue --
-        const int ew = warp - 6;           // 0..7
-        const int q = warp & 3;            // TMEM lane quadrant this warp may access
-        const int hcol = ew >> 2;          // column half
-        const int r = q * 32 + lane;       // A row = weight column within the tile
+        const int ew = warp - kUnpackWarps;  // 0..7
+        const int q = warp & 3;              // TMEM lane quadrant this warp may access
+        const int hcol = ew >> 2;            // column half
+        const int r = q * 32 + lane;         // weight row within the tile
         constexpr int CH = C::CH;
         const uint32_t lane_addr = ((uint32_t)(q * 32)) << 16;
 
-        // Pre-fill both partial buffers, then hand them to the MMA warp.
+        // Arm every partial buffer, then hand them to the MMA warp.
 #pragma unroll
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < NACC; ++b) {
             const uint32_t ta = tmem_base + lane_addr + b * BN + hcol * CH;
             if constexpr (CH >= 32) {
 #pragma unroll
@@ -406,13 +440,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) {
-            mbar_arrive(&acc_empty[0]);
-            mbar_arrive(&acc_empty[1]);
-        }
+        if (lane == 0)
+            for (int b = 0; b < NACC; ++b) mbar_arrive(&acc_empty[b]);
 
-        Ring ac;
         bool ok = true;
+        Ring rw, rc;
         for (long long u = u0; u < u1 && ok;) {
             const long long t = u / G;
             const int gb = (int)(u % G);
@@ -423,19 +455,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const int half = r >> 6;
             const bool n_valid = (half == 0) || (nb1 >= 0);
             const int n = (half == 0 ? nb0 : nb1) * 64 + (r & 63);  // weight column
-            const float* swp = p.s_w + (long long)ti.e * p.sw_estride + n;
 
             float acc[CH];
 #pragma unroll
-            for (int j = 0; j < CH; ++j) acc[j] = 0.0f;
-            float sw_next = n_valid ? __ldg(swp + (long long)gb * p.N) : 0.0f;
+            for (int jj = 0; jj < CH; ++jj) acc[jj] = 0.0f;
 
-            for (int gi = gb; gi < ge; ++gi) {
-                const float sw = sw_next;
-                if (gi + 1 < ge) sw_next = n_valid ? __ldg(swp + (long long)(gi + 1) * p.N) : 0.0f;
-                if (!warp_wait_bounded(&acc_full[ac.idx], ac.phase, wc)) { ok = false; break; }
+            for (int gi = gb; gi < ge; ++gi, rw.next(C::SWS), rc.next(NACC)) {
+                const uint32_t w = rw.idx;
+                if (!warp_wait_bounded(&sw_full[w], rw.phase, wc)) { ok = false; break; }
+                const float sw = n_valid ? sSW[w * 128 + r] : 0.0f;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sw_empty[w]);
+                const uint32_t ab = rc.idx;
+                if (!warp_wait_bounded(&acc_full[ab], rc.phase, wc)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t ta = tmem_base + lane_addr + ac.idx * BN + hcol * CH;
+                const uint32_t ta = tmem_base + lane_addr + ab * BN + hcol * CH;
                 constexpr int CW = CH < 16 ? CH : 16;  // columns per TMEM load
 #pragma unroll
                 for (int c0 = 0; c0 < CH; c0 += CW) {
@@ -444,15 +478,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     tmem_wait_ld();
                     tmem_fill32<CW>(ta + c0, kMagicBits);  // re-arm for the next group
 #pragma unroll
-                    for (int j = 0; j < CW; ++j)
-                        acc[c0 + j] = fmaf(sw, __uint_as_float(v[j]) - kMagicF, acc[c0 + j]);
+                    for (int jj = 0; jj < CW; ++jj)
+                        acc[c0 + jj] = fmaf(sw, __uint_as_float(v[jj]) - kMagicF, acc[c0 + jj]);
                     if (p.dbgP != nullptr && n_valid) {
 #pragma unroll
-                        for (int j = 0; j < CW; ++j) {
-                            const int col = hcol * CH + c0 + j;
+                        for (int jj = 0; jj < CW; ++jj) {
+                            const int col = hcol * CH + c0 + jj;
                             if (col < ti.rows_valid) {
                                 const long long m = ti.row0 + col;
-                                p.dbgP[(m * G + gi) * p.N + n] = (int32_t)(v[j] - kMagicBits);
+                                p.dbgP[(m * G + gi) * p.N + n] = (int32_t)(v[jj] - kMagicBits);
                             }
                         }
                     }
@@ -460,8 +494,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&acc_empty[ac.idx]);
-                ac.next(2);
+                if (lane == 0) mbar_arrive(&acc_empty[ab]);
             }
             if (p.mode == kModeGateUp) {
                 // The exchange below uses named barriers: decide together
@@ -478,40 +511,40 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 const long long slot = (long long)blockIdx.x - c_first;
                 float* dst = p.partial + ((t * p.slots + slot) * BN) * 128 + r;
 #pragma unroll
-                for (int j = 0; j < CH; ++j) dst[(long long)(hcol * CH + j) * 128] = acc[j];
+                for (int jj = 0; jj < CH; ++jj) dst[(long long)(hcol * CH + jj) * 128] = acc[jj];
             } else if (p.mode == kModeGateUp) {
                 // rows 64..127 hold "up", rows 0..63 the matching "gate"
                 if (half == 1) {
 #pragma unroll
-                    for (int j = 0; j < CH; ++j) {
-                        const int col = hcol * CH + j;
+                    for (int jj = 0; jj < CH; ++jj) {
+                        const int col = hcol * CH + jj;
                         const float sx = (col < ti.rows_valid) ? __ldg(p.s_x + ti.row0 + col) : 0.0f;
-                        sX[col * 64 + (r - 64)] = sx * acc[j];
+                        sX[col * 64 + (r - 64)] = sx * acc[jj];
                     }
                 }
                 named_bar_sync(1, kNumEpiWarps * 32);
                 if (half == 0) {
-                    const int i = ti.nt * 64 + r;
+                    const int ii = ti.nt * 64 + r;
 #pragma unroll
-                    for (int j = 0; j < CH; ++j) {
-                        const int col = hcol * CH + j;
+                    for (int jj = 0; jj < CH; ++jj) {
+                        const int col = hcol * CH + jj;
                         if (col < ti.rows_valid) {
                             const long long m = ti.row0 + col;
-                            const float gte = __ldg(p.s_x + m) * acc[j];
+                            const float gte = __ldg(p.s_x + m) * acc[jj];
                             const float up = sX[col * 64 + r];
                             const float hv = (gte / (1.0f + expf(-gte))) * up;
-                            p.Y[m * p.ldy + i] = f32_to_bf16_bits(hv);
+                            p.Y[m * p.ldy + ii] = f32_to_bf16_bits(hv);
                         }
                     }
                 }
                 named_bar_sync(1, kNumEpiWarps * 32);
             } else if (full_tile && n_valid) {
 #pragma unroll
-                for (int j = 0; j < CH; ++j) {
-                    const int col = hcol * CH + j;
+                for (int jj = 0; jj < CH; ++jj) {
+                    const int col = hcol * CH + jj;
                     if (col < ti.rows_valid) {
                         const long long m = ti.row0 + col;
-                        p.Y[m * p.ldy + n] = f32_to_bf16_bits(__ldg(p.s_x + m) * acc[j]);
+                        p.Y[m * p.ldy + n] = f32_to_bf16_bits(__ldg(p.s_x + m) * acc[jj]);
                     }
                 }
             }
@@ -522,7 +555,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ----------------------------------------------------------- teardown --
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == kWarpMma) {
         tc_fence_after();
         tmem_dealloc(tmem_base, C::TMEM_COLS);
     }

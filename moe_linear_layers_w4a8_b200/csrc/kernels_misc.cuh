@@ -405,7 +405,7 @@ __global__ void bounded_wait_selftest_kernel(int32_t* status, unsigned long long
         fence_mbar_init();
     }
     __syncthreads();
-    WaitCtx w{&abort_flag, status, limit_ns};
+    WaitCtx w{&abort_flag, status, wait_cycles_for_ns(limit_ns)};
     if (threadIdx.x == 0) (void)wait_bounded(&bar, 0, w);
     __syncthreads();
 }

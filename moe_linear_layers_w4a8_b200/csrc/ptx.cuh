@@ -12,12 +12,6 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-__device__ __forceinline__ uint64_t globaltimer_ns() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
 // ------------------------------------------------------------ mbarrier --
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
@@ -53,35 +47,54 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Like mbar_try_wait, but a thread whose phase is not complete yet sleeps
+// (until the phase completes, or at most about `hint_ns`) instead of
+// returning at once, so waiting warps do not take issue slots from the
+// warps doing work.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Shared context of the bounded waits of one CTA.  `abort` lives in shared
 // memory: once any wait gives up, every other wait of the CTA returns false
 // promptly so that all roles reach the common exit.
 struct WaitCtx {
     volatile int* abort;
-    int32_t* status;      // device status word of the call (may be null)
-    uint64_t limit_ns;    // per-wait limit
+    int32_t* status;        // device status word of the call (may be null)
+    long long limit_cycles; // per-wait limit in SM clock cycles
 };
 
 __device__ __forceinline__ void report_status(int32_t* status, int code) {
     if (status) atomicCAS(reinterpret_cast<int*>(status), 0, code);
 }
 
+// SM cycles that cover `ns` nanoseconds at any SM clock up to 2 GHz.
+__host__ __device__ constexpr long long wait_cycles_for_ns(unsigned long long ns) {
+    return (long long)(ns * 2ull);
+}
+
 // Waits for the phase of `bar` with the given parity to complete.  Returns
-// false (after recording W4A8_ERR_TIMEOUT = 5) if `limit_ns` elapses, or if
-// another wait of the CTA already gave up.
+// false (after recording W4A8_ERR_TIMEOUT = 5) once `limit_cycles` SM cycles
+// have passed, or when another wait of the CTA already gave up.  The SM
+// cycle counter is cheap to read, so the common path costs one try_wait.
 __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
     if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = globaltimer_ns();
-    uint32_t n = 0;
+    const long long t0 = clock64();
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((++n & 15u) == 0u) {
-            if (*w.abort) return false;
-            if (globaltimer_ns() - t0 > w.limit_ns) {
-                *w.abort = 1;
-                report_status(w.status, 5);
-                return false;
-            }
+        if (mbar_try_wait_sleep(bar, parity, 100000u)) return true;  // sleeps <= ~0.1 ms
+        if (*w.abort) return false;
+        if (clock64() - t0 > w.limit_cycles) {
+            *w.abort = 1;
+            report_status(w.status, 5);
+            return false;
         }
     }
 }
@@ -156,6 +169,18 @@ __device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t
         : "memory");
 }
 
+// D[tmem] (+)= A[tmem] * B[smem]^T, signed int8 x signed int8 -> int32; the
+// A tile sits in TMEM (lane = row, 4 consecutive k per 32-bit column).
+__device__ __forceinline__ void mma_i8_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                              uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Shared-memory matrix descriptor of a K-major operand tile whose rows are
 // `row_bytes` (64 or 128) long and swizzled with the matching 64B / 128B
 // pattern (8-row atoms, atom stride 8 * row_bytes).
@@ -207,6 +232,32 @@ __device__ __forceinline__ void tmem_ld32<32>(uint32_t taddr, uint32_t* r) {
           "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]),
           "=r"(r[30]), "=r"(r[31])
         : "r"(taddr));
+}
+
+// Registers -> TMEM, 32 lanes x N consecutive 32-bit columns.
+template <int N>
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r);
+
+template <>
+__device__ __forceinline__ void tmem_st32<16>(uint32_t taddr, const uint32_t* r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+            taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+
+template <>
+__device__ __forceinline__ void tmem_st32<32>(uint32_t taddr, const uint32_t* r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+        "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+        "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
 }
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }

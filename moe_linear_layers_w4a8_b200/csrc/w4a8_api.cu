@@ -77,22 +77,25 @@ w4a8_status last_cuda() { return cudaGetLastError() == cudaSuccess ? W4A8_OK : W
 
 // ---------------------------------------------------------- GEMM configs --
 
+// Ring depths: SP packed-code stages (shared memory), SA activation +
+// unpacked-weight stages (shared memory + TMEM), NACC TMEM partial buffers.
+// TMEM columns used: NACC * BN + SA * GROUP / 4 <= 512.
 template <int BN, int GROUP>
 struct Stages;
-template <> struct Stages<16, 128> { static constexpr int S = 12, SA = 3; };
-template <> struct Stages<32, 128> { static constexpr int S = 10, SA = 3; };
-template <> struct Stages<64, 128> { static constexpr int S = 8, SA = 3; };
-template <> struct Stages<128, 128> { static constexpr int S = 5, SA = 3; };
-template <> struct Stages<16, 64> { static constexpr int S = 16, SA = 4; };
-template <> struct Stages<32, 64> { static constexpr int S = 16, SA = 4; };
-template <> struct Stages<64, 64> { static constexpr int S = 12, SA = 4; };
-template <> struct Stages<128, 64> { static constexpr int S = 8, SA = 4; };
+template <> struct Stages<16, 128> { static constexpr int SP = 20, SA = 8, NACC = 8; };
+template <> struct Stages<32, 128> { static constexpr int SP = 16, SA = 8, NACC = 8; };
+template <> struct Stages<64, 128> { static constexpr int SP = 12, SA = 8, NACC = 4; };
+template <> struct Stages<128, 128> { static constexpr int SP = 12, SA = 4, NACC = 3; };
+template <> struct Stages<16, 64> { static constexpr int SP = 32, SA = 8, NACC = 8; };
+template <> struct Stages<32, 64> { static constexpr int SP = 24, SA = 8, NACC = 8; };
+template <> struct Stages<64, 64> { static constexpr int SP = 24, SA = 8, NACC = 6; };
+template <> struct Stages<128, 64> { static constexpr int SP = 16, SA = 8, NACC = 3; };
 
 template <int BN, int GROUP>
 w4a8_status launch_gemm_t(const CUtensorMap& tmap, const GemmParams& p, int grid, cudaStream_t stream) {
-    constexpr int S = Stages<BN, GROUP>::S, SA = Stages<BN, GROUP>::SA;
-    using C = GemmCfg<BN, GROUP, S, SA>;
-    auto kern = w4a8_gemm_tc_kernel<BN, GROUP, S, SA>;
+    constexpr int SP = Stages<BN, GROUP>::SP, SA = Stages<BN, GROUP>::SA, NACC = Stages<BN, GROUP>::NACC;
+    using C = GemmCfg<BN, GROUP, SP, SA, NACC>;
+    auto kern = w4a8_gemm_tc_kernel<BN, GROUP, SP, SA, NACC>;
     static std::atomic<uint64_t> attr_done{0};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -392,12 +395,13 @@ w4a8_status w4a8_gemm_debug_partials(const int8_t* qx, const float* s_x, const u
     return gemm_impl(qx, s_x, packed, s_w, z, w, M, Y, ldy, P, workspace, ws_bytes, dev_status, stream);
 }
 
-w4a8_status w4a8_moe_grouped_gemm(const uint16_t* X, const float* logits, int T, int E, int topk,
-                                  const uint8_t* w1_packed, const float* w1_s, const uint8_t* w1_z,
-                                  const w4a8_wdesc* w1, const uint8_t* w2_packed, const float* w2_s,
-                                  const uint8_t* w2_z, const w4a8_wdesc* w2, uint16_t* out,
-                                  int32_t* topk_idx_out, float* topk_w_out, int32_t* expert_offsets_out,
-                                  void* workspace, size_t ws_bytes, int32_t* dev_status, void* stream) {
+w4a8_status w4a8_moe_grouped_gemm_profiled(const uint16_t* X, const float* logits, int T, int E, int topk,
+                                           const uint8_t* w1_packed, const float* w1_s, const uint8_t* w1_z,
+                                           const w4a8_wdesc* w1, const uint8_t* w2_packed, const float* w2_s,
+                                           const uint8_t* w2_z, const w4a8_wdesc* w2, uint16_t* out,
+                                           int32_t* topk_idx_out, float* topk_w_out, int32_t* expert_offsets_out,
+                                           void* workspace, size_t ws_bytes, int32_t* dev_status, void* stream,
+                                           void* const* stage_events) {
     w4a8_status st = check_moe(T, E, topk, w1, w2);
     if (st != W4A8_OK) return st;
     if (T == 0) return W4A8_OK;
@@ -428,8 +432,14 @@ w4a8_status w4a8_moe_grouped_gemm(const uint16_t* X, const float* logits, int T,
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int R = T * topk;
     const int bn = pick_bn(((long long)R + E - 1) / E);
+    auto mark = [&](int i) -> bool {
+        if (!stage_events || !stage_events[i]) return true;
+        return cudaEventRecordWithFlags(static_cast<cudaEvent_t>(stage_events[i]), s, cudaEventRecordExternal) ==
+               cudaSuccess;
+    };
 
     // 1. routing
+    if (!mark(0)) return W4A8_ERR_CUDA;
     {
         const int epl = (E + 31) / 32;
         const unsigned blocks = (unsigned)(((long long)T * 32 + 255) / 256);
@@ -444,12 +454,15 @@ w4a8_status w4a8_moe_grouped_gemm(const uint16_t* X, const float* logits, int T,
         if ((st = last_cuda()) != W4A8_OK) return st;
     }
     // 2. dispatch
+    if (!mark(1)) return W4A8_ERR_CUDA;
     dispatch_kernel<<<1, kDispatchThreads, 0, s>>>(topk_idx_out, T, E, topk, bn, expert_offsets_out, mtile_off,
                                                    perm, inv);
     if ((st = last_cuda()) != W4A8_OK) return st;
     // 3. quantize X straight into dispatch order
+    if (!mark(2)) return W4A8_ERR_CUDA;
     if ((st = launch_quant(X, T, H, H, qx, sx, nullptr, 0, inv, topk, dev_status, s)) != W4A8_OK) return st;
     // 4. gate_up + SiLU * up
+    if (!mark(3)) return W4A8_ERR_CUDA;
     {
         CUtensorMap tmap;
         if (!make_act_tmap(&tmap, qx, R, H, group, bn)) return W4A8_ERR_CUDA;
@@ -477,8 +490,10 @@ w4a8_status w4a8_moe_grouped_gemm(const uint16_t* X, const float* logits, int T,
         if ((st = launch_gemm(bn, group, tmap, p, sms, s)) != W4A8_OK) return st;
     }
     // 5. quantize h per (token, expert) row
+    if (!mark(4)) return W4A8_ERR_CUDA;
     if ((st = launch_quant(h, R, I, I, qh, sh, nullptr, 0, nullptr, 0, dev_status, s)) != W4A8_OK) return st;
     // 6. down
+    if (!mark(5)) return W4A8_ERR_CUDA;
     {
         CUtensorMap tmap;
         if (!make_act_tmap(&tmap, qh, R, I, group, bn)) return W4A8_ERR_CUDA;
@@ -505,12 +520,25 @@ w4a8_status w4a8_moe_grouped_gemm(const uint16_t* X, const float* logits, int T,
         if ((st = launch_gemm(bn, group, tmap, p, sms, s)) != W4A8_OK) return st;
     }
     // 7. weighted combine
+    if (!mark(6)) return W4A8_ERR_CUDA;
     {
         const long long n = (long long)T * (H / 8);
         combine_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(yd, topk_w_out, inv, T, topk, H, out);
         if ((st = last_cuda()) != W4A8_OK) return st;
     }
+    if (!mark(7)) return W4A8_ERR_CUDA;
     return W4A8_OK;
+}
+
+w4a8_status w4a8_moe_grouped_gemm(const uint16_t* X, const float* logits, int T, int E, int topk,
+                                  const uint8_t* w1_packed, const float* w1_s, const uint8_t* w1_z,
+                                  const w4a8_wdesc* w1, const uint8_t* w2_packed, const float* w2_s,
+                                  const uint8_t* w2_z, const w4a8_wdesc* w2, uint16_t* out,
+                                  int32_t* topk_idx_out, float* topk_w_out, int32_t* expert_offsets_out,
+                                  void* workspace, size_t ws_bytes, int32_t* dev_status, void* stream) {
+    return w4a8_moe_grouped_gemm_profiled(X, logits, T, E, topk, w1_packed, w1_s, w1_z, w1, w2_packed, w2_s, w2_z,
+                                          w2, out, topk_idx_out, topk_w_out, expert_offsets_out, workspace,
+                                          ws_bytes, dev_status, stream, nullptr);
 }
 
 w4a8_status w4a8_get_device_status(const int32_t* dev_status, void* stream) {
