@@ -10,9 +10,11 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libw4a8.so")
-SOURCES = [os.path.join(CSRC, "w4a8_api.cu")]
+SOURCES = [os.path.join(CSRC, f) for f in
+           ("w4a8_api.cu", "gemm_plain.cu", "gemm_splitk.cu", "gemm_gateup.cu", "gemm_down.cu")]
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")] + [
     os.path.join(INCLUDE, "w4a8.h")]
+BUILD_DIR = os.path.join(PKG, "_build")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -35,13 +37,26 @@ def needs_build() -> bool:
 
 
 def build(force: bool = False, verbose_ptxas: bool = False) -> str:
+    """Compiles every translation unit in parallel, then links libw4a8.so."""
     if not force and not needs_build():
         return LIB
+    os.makedirs(BUILD_DIR, exist_ok=True)
+    compile_flags = [f for f in NVCC_FLAGS if f != "-shared"]
+    procs, objs = [], []
+    for src in SOURCES:
+        obj = os.path.join(BUILD_DIR, os.path.basename(src) + f".{os.getpid()}.o")
+        cmd = [nvcc(), *compile_flags, "-c", "-I", INCLUDE, "-I", CSRC, src, "-o", obj]
+        if verbose_ptxas:
+            cmd += ["-Xptxas", "-v"]
+        procs.append((src, subprocess.Popen(cmd)))
+        objs.append(obj)
+    failed = [src for src, pr in procs if pr.wait() != 0]
+    if failed:
+        raise RuntimeError(f"nvcc failed on {failed}")
     tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, *SOURCES, "-o", tmp]
-    if verbose_ptxas:
-        cmd += ["-Xptxas", "-v"]
-    subprocess.check_call(cmd)
+    subprocess.check_call([nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", *objs, "-o", tmp])
+    for o in objs:
+        os.remove(o)
     os.replace(tmp, LIB)
     return LIB
 

@@ -1,0 +1,11 @@
+// Instantiations of the W4A8 GEMM kernel for the gateup output mode.
+#include "gemm_launch.cuh"
+
+namespace w4a8 {
+
+int launch_gemm_gateup(int bn, int group, const CUtensorMap& tmap, const GemmParams& p, int grid,
+                      cudaStream_t stream) {
+    return launch_gemm_mode<kModeGateUp, false>(bn, group, tmap, p, grid, stream);
+}
+
+}  // namespace w4a8

@@ -40,7 +40,6 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
-#include "kernels_misc.cuh"
 #include "ptx.cuh"
 
 namespace w4a8 {
@@ -131,12 +130,12 @@ struct TileInfo {
     int rows_valid;  // activation rows of this tile that exist
 };
 
-template <int BN>
+template <int BN, int MODE>
 __device__ __forceinline__ TileInfo decode_tile(const GemmParams& p, long long t) {
     TileInfo ti;
     const int gm = (int)(t / p.n_tiles);
     ti.nt = (int)(t % p.n_tiles);
-    if (p.mode == kModeGateUp || p.mode == kModeDown) {
+    if constexpr (MODE == kModeGateUp || MODE == kModeDown) {
         int lo = 0, hi = p.E - 1;  // last expert whose m-tile prefix is <= gm
         while (lo < hi) {
             const int mid = (lo + hi + 1) >> 1;
@@ -159,8 +158,9 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmParams& p, long long t
 
 // 64-column weight blocks that form the 128 A rows of a tile: rows 0..63
 // come from block nb0 and rows 64..127 from block nb1 (nb1 < 0: absent).
+template <int MODE>
 __device__ __forceinline__ void tile_blocks(const GemmParams& p, int nt, int& nb0, int& nb1) {
-    if (p.mode == kModeGateUp) {
+    if constexpr (MODE == kModeGateUp) {
         nb0 = nt;                  // gate columns [64 nt, 64 nt + 64)
         nb1 = (p.I >> 6) + nt;     // matching up columns I + [64 nt, ...)
     } else {
@@ -170,9 +170,10 @@ __device__ __forceinline__ void tile_blocks(const GemmParams& p, int nt, int& nb
 }
 
 // Work range of this CTA in (tile, group) units.
+template <int MODE>
 __device__ __forceinline__ void cta_units(const GemmParams& p, long long& u0, long long& u1, long long& Q) {
     long long U;
-    if (p.mode == kModeGateUp || p.mode == kModeDown) {
+    if constexpr (MODE == kModeGateUp || MODE == kModeDown) {
         const long long tiles = (long long)__ldg(p.mtile_off + p.E) * p.n_tiles;
         U = tiles * p.G;
         Q = (long long)p.G * ((tiles + gridDim.x - 1) / gridDim.x);
@@ -189,7 +190,9 @@ constexpr int kUnpackWarps = 4;
 
 constexpr int kWarpPack = 12, kWarpAct = 13, kWarpMma = 14;
 
-template <int BN, int GROUP, int SP, int SA, int NACC>
+// MODE (GemmMode) and DBG (write the int32 group partials) are compile-time,
+// so each launched kernel carries only its own epilogue.
+template <int BN, int GROUP, int SP, int SA, int NACC, int MODE, bool DBG>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     w4a8_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act, const GemmParams p) {
     using C = GemmCfg<BN, GROUP, SP, SA, NACC>;
@@ -252,7 +255,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const WaitCtx wc{abort_flag, p.status, wait_cycles_for_ns(p.wait_ns)};
 
     long long u0, u1, Q;
-    cta_units(p, u0, u1, Q);
+    cta_units<MODE>(p, u0, u1, Q);
     const int G = p.G;
     const long long nsteps = u1 - u0;  // one step = one K-group of one tile
 
@@ -271,8 +274,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             Ring rs, rw;  // this producer's ring; s_w ring (activation producer)
             for (long long i = 0; i < nsteps; ++i) {
                 if (t != cur_t) {
-                    ti = decode_tile<BN>(p, t);
-                    tile_blocks(p, ti.nt, nb0, nb1);
+                    ti = decode_tile<BN, MODE>(p, t);
+                    tile_blocks<MODE>(p, ti.nt, nb0, nb1);
                     cur_t = t;
                 }
                 const uint32_t s = rs.idx;
@@ -377,9 +380,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         Ring rp, ra;
         for (long long i = 0; i < nsteps; ++i, rp.next(SP), ra.next(SA)) {
             if (t != cur_t) {
-                const TileInfo ti = decode_tile<BN>(p, t);
+                const TileInfo ti = decode_tile<BN, MODE>(p, t);
                 int nb0;
-                tile_blocks(p, ti.nt, nb0, nb1);
+                tile_blocks<MODE>(p, ti.nt, nb0, nb1);
                 cur_t = t;
             }
             if (++gi == G) { gi = 0; ++t; }
@@ -449,9 +452,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const long long t = u / G;
             const int gb = (int)(u % G);
             const int ge = (int)min((long long)G, gb + (u1 - u));
-            const TileInfo ti = decode_tile<BN>(p, t);
+            const TileInfo ti = decode_tile<BN, MODE>(p, t);
             int nb0, nb1;
-            tile_blocks(p, ti.nt, nb0, nb1);
+            tile_blocks<MODE>(p, ti.nt, nb0, nb1);
             const int half = r >> 6;
             const bool n_valid = (half == 0) || (nb1 >= 0);
             const int n = (half == 0 ? nb0 : nb1) * 64 + (r & 63);  // weight column
@@ -480,7 +483,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
                     for (int jj = 0; jj < CW; ++jj)
                         acc[c0 + jj] = fmaf(sw, __uint_as_float(v[jj]) - kMagicF, acc[c0 + jj]);
-                    if (p.dbgP != nullptr && n_valid) {
+                    if (DBG && n_valid) {
 #pragma unroll
                         for (int jj = 0; jj < CW; ++jj) {
                             const int col = hcol * CH + c0 + jj;
@@ -496,7 +499,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&acc_empty[ab]);
             }
-            if (p.mode == kModeGateUp) {
+            if constexpr (MODE == kModeGateUp) {
                 // The exchange below uses named barriers: decide together
                 // whether any epilogue warp gave up, so none waits alone.
                 if (named_bar_or(2, kNumEpiWarps * 32, !ok)) break;
@@ -506,13 +509,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
             // ---------------------------------------------- tile output --
             const bool full_tile = (gb == 0 && ge == G);
-            if (p.mode == kModeSplitK) {
+            if constexpr (MODE == kModeSplitK) {
                 const long long c_first = (t * G) / Q;
                 const long long slot = (long long)blockIdx.x - c_first;
                 float* dst = p.partial + ((t * p.slots + slot) * BN) * 128 + r;
 #pragma unroll
                 for (int jj = 0; jj < CH; ++jj) dst[(long long)(hcol * CH + jj) * 128] = acc[jj];
-            } else if (p.mode == kModeGateUp) {
+            } else if constexpr (MODE == kModeGateUp) {
                 // rows 64..127 hold "up", rows 0..63 the matching "gate"
                 if (half == 1) {
 #pragma unroll
@@ -538,13 +541,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     }
                 }
                 named_bar_sync(1, kNumEpiWarps * 32);
-            } else if (full_tile && n_valid) {
+            } else {
+                if (full_tile && n_valid) {
 #pragma unroll
-                for (int jj = 0; jj < CH; ++jj) {
-                    const int col = hcol * CH + jj;
-                    if (col < ti.rows_valid) {
-                        const long long m = ti.row0 + col;
-                        p.Y[m * p.ldy + n] = f32_to_bf16_bits(__ldg(p.s_x + m) * acc[jj]);
+                    for (int jj = 0; jj < CH; ++jj) {
+                        const int col = hcol * CH + jj;
+                        if (col < ti.rows_valid) {
+                            const long long m = ti.row0 + col;
+                            p.Y[m * p.ldy + n] = f32_to_bf16_bits(__ldg(p.s_x + m) * acc[jj]);
+                        }
                     }
                 }
             }

@@ -12,13 +12,6 @@ namespace w4a8 {
 
 constexpr int kStatusNonfinite = 4;
 
-__device__ __forceinline__ float bf16_bits_to_f32(uint32_t h16) { return __uint_as_float(h16 << 16); }
-
-__device__ __forceinline__ uint16_t f32_to_bf16_bits(float f) {
-    __nv_bfloat16 b = __float2bfloat16_rn(f);
-    return *reinterpret_cast<uint16_t*>(&b);
-}
-
 // ---------------------------------------------------------------------------
 // Per-token INT8 activation quantization ("Inference Quantization ch.1" §9.2;
 // "Kimi 2.7 MoE, 4-bit storage to INT8" §3.3):

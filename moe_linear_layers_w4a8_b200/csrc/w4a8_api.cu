@@ -12,7 +12,7 @@
 #include <mutex>
 
 #include "w4a8.h"
-#include "gemm_tc.cuh"
+#include "gemm_launch.cuh"
 #include "kernels_misc.cuh"
 
 using namespace w4a8;
@@ -77,56 +77,18 @@ w4a8_status last_cuda() { return cudaGetLastError() == cudaSuccess ? W4A8_OK : W
 
 // ---------------------------------------------------------- GEMM configs --
 
-// Ring depths: SP packed-code stages (shared memory), SA activation +
-// unpacked-weight stages (shared memory + TMEM), NACC TMEM partial buffers.
-// TMEM columns used: NACC * BN + SA * GROUP / 4 <= 512.
-template <int BN, int GROUP>
-struct Stages;
-template <> struct Stages<16, 128> { static constexpr int SP = 20, SA = 8, NACC = 8; };
-template <> struct Stages<32, 128> { static constexpr int SP = 16, SA = 8, NACC = 8; };
-template <> struct Stages<64, 128> { static constexpr int SP = 12, SA = 8, NACC = 4; };
-template <> struct Stages<128, 128> { static constexpr int SP = 12, SA = 4, NACC = 3; };
-template <> struct Stages<16, 64> { static constexpr int SP = 32, SA = 8, NACC = 8; };
-template <> struct Stages<32, 64> { static constexpr int SP = 24, SA = 8, NACC = 8; };
-template <> struct Stages<64, 64> { static constexpr int SP = 24, SA = 8, NACC = 6; };
-template <> struct Stages<128, 64> { static constexpr int SP = 16, SA = 8, NACC = 3; };
-
-template <int BN, int GROUP>
-w4a8_status launch_gemm_t(const CUtensorMap& tmap, const GemmParams& p, int grid, cudaStream_t stream) {
-    constexpr int SP = Stages<BN, GROUP>::SP, SA = Stages<BN, GROUP>::SA, NACC = Stages<BN, GROUP>::NACC;
-    using C = GemmCfg<BN, GROUP, SP, SA, NACC>;
-    auto kern = w4a8_gemm_tc_kernel<BN, GROUP, SP, SA, NACC>;
-    static std::atomic<uint64_t> attr_done{0};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    const uint64_t bit = 1ull << (dev & 63);
-    if (!(attr_done.load() & bit)) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
-            return W4A8_ERR_CUDA;
-        attr_done.fetch_or(bit);
+// GEMM launch: per-mode entry points live in gemm_<mode>.cu (see gemm_launch.cuh).
+w4a8_status launch_gemm(int mode, bool dbg, int bn, int group, const CUtensorMap& tmap, const GemmParams& p,
+                        int grid, cudaStream_t stream) {
+    int r;
+    switch (mode) {
+        case kModePlain: r = launch_gemm_plain(dbg, bn, group, tmap, p, grid, stream); break;
+        case kModeSplitK: r = launch_gemm_splitk(dbg, bn, group, tmap, p, grid, stream); break;
+        case kModeGateUp: r = launch_gemm_gateup(bn, group, tmap, p, grid, stream); break;
+        case kModeDown: r = launch_gemm_down(bn, group, tmap, p, grid, stream); break;
+        default: r = W4A8_ERR_UNSUPPORTED_SHAPE;
     }
-    kern<<<grid, kGemmThreads, C::SMEM, stream>>>(tmap, p);
-    return last_cuda();
-}
-
-w4a8_status launch_gemm(int bn, int group, const CUtensorMap& tmap, const GemmParams& p, int grid,
-                        cudaStream_t stream) {
-    if (group == 128) {
-        switch (bn) {
-            case 16: return launch_gemm_t<16, 128>(tmap, p, grid, stream);
-            case 32: return launch_gemm_t<32, 128>(tmap, p, grid, stream);
-            case 64: return launch_gemm_t<64, 128>(tmap, p, grid, stream);
-            case 128: return launch_gemm_t<128, 128>(tmap, p, grid, stream);
-        }
-    } else {
-        switch (bn) {
-            case 16: return launch_gemm_t<16, 64>(tmap, p, grid, stream);
-            case 32: return launch_gemm_t<32, 64>(tmap, p, grid, stream);
-            case 64: return launch_gemm_t<64, 64>(tmap, p, grid, stream);
-            case 128: return launch_gemm_t<128, 64>(tmap, p, grid, stream);
-        }
-    }
-    return W4A8_ERR_UNSUPPORTED_SHAPE;
+    return static_cast<w4a8_status>(r);
 }
 
 int pick_bn(long long rows_per_group) {
@@ -217,7 +179,7 @@ w4a8_status gemm_impl(const int8_t* qx, const float* s_x, const uint8_t* packed,
     p.status = dev_status;
     p.wait_ns = kDefaultWaitNs;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    st = launch_gemm(pl.bn, w->group, tmap, p, pl.grid, s);
+    st = launch_gemm(p.mode, P != nullptr, pl.bn, w->group, tmap, p, pl.grid, s);
     if (st != W4A8_OK) return st;
     if (pl.splitk) {
         const long long n = (long long)M * w->N;
@@ -487,7 +449,7 @@ w4a8_status w4a8_moe_grouped_gemm_profiled(const uint16_t* X, const float* logit
         p.I = I;
         p.status = dev_status;
         p.wait_ns = kDefaultWaitNs;
-        if ((st = launch_gemm(bn, group, tmap, p, sms, s)) != W4A8_OK) return st;
+        if ((st = launch_gemm(kModeGateUp, false, bn, group, tmap, p, sms, s)) != W4A8_OK) return st;
     }
     // 5. quantize h per (token, expert) row
     if (!mark(4)) return W4A8_ERR_CUDA;
@@ -517,7 +479,7 @@ w4a8_status w4a8_moe_grouped_gemm_profiled(const uint16_t* X, const float* logit
         p.E = E;
         p.status = dev_status;
         p.wait_ns = kDefaultWaitNs;
-        if ((st = launch_gemm(bn, group, tmap, p, sms, s)) != W4A8_OK) return st;
+        if ((st = launch_gemm(kModeDown, false, bn, group, tmap, p, sms, s)) != W4A8_OK) return st;
     }
     // 7. weighted combine
     if (!mark(6)) return W4A8_ERR_CUDA;
