@@ -3,10 +3,10 @@
 
 namespace w4a8 {
 
-int launch_gemm_splitk(bool dbg, int bn, int group, const CUtensorMap& tmap, const GemmParams& p, int grid,
+int launch_gemm_splitk(bool dbg, int bn, int group, const GemmMaps& maps, const GemmParams& p, int grid,
                       cudaStream_t stream) {
-    return dbg ? launch_gemm_mode<kModeSplitK, true>(bn, group, tmap, p, grid, stream)
-               : launch_gemm_mode<kModeSplitK, false>(bn, group, tmap, p, grid, stream);
+    return dbg ? launch_gemm_mode<kModeSplitK, true>(bn, group, maps, p, grid, stream)
+               : launch_gemm_mode<kModeSplitK, false>(bn, group, maps, p, grid, stream);
 }
 
 }  // namespace w4a8

@@ -27,7 +27,13 @@
 //     0x4B400000 before a group's MMAs, so afterwards it holds the bits of
 //     the float 12582912 + P (|P| < 2^22): one FADD turns it into P exactly,
 //     one FFMA applies s_w.
-//   * K is walked one quantization group per pipeline step.
+//   * K is walked one quantization group per MMA step, but every TMA request
+//     brings several consecutive groups ("chunks"): the packed codes of up to
+//     4 (g=128) / 8 (g=64) groups per 64-column half, the activation tiles of
+//     up to 8 groups through a 3-D tensor map (k within group, row, group),
+//     and the scales / zero-points of 8 groups through 2-D tensor maps.  An
+//     SM's TMA unit spends a roughly fixed time per request, so few large
+//     requests keep it off the critical path.
 //   * Persistent: each CTA owns a contiguous range of (tile, group) units.
 //     Ranges that split a tile (split-K) write fp32 partial tiles that a
 //     second kernel sums in a fixed order.
@@ -77,39 +83,48 @@ constexpr int kNumEpiWarps = 8;
 constexpr uint32_t kMagicBits = 0x4B400000u;  // float 12582912 = 1.5 * 2^23
 constexpr float kMagicF = 12582912.0f;
 
-template <int BN, int GROUP, int SP, int SA, int NACC_>
+// Ring geometry of one kernel instantiation.
+template <int BN, int GROUP, int MODE>
 struct GemmCfg {
-    // P ring: packed codes + zero-points (TMA -> unpack warps).
-    // A ring: activation tile (TMA, shared memory) + unpacked weight tile
-    //         (unpack warps, TMEM), both drained by the MMA.
-    static constexpr int NACC = NACC_;           // TMEM partial buffers
-    static constexpr int GW = GROUP / 4;         // TMEM columns of one unpacked group
-    static constexpr int A_COL0 = NACC * BN;     // first TMEM column of the A ring
-    static constexpr int ACT_STAGE = BN * GROUP;
-    static constexpr int PK_HALF = 32 * GROUP;   // one 64-column block of one group
-    static constexpr int PK_STAGE = 2 * PK_HALF;
-    static constexpr int Z_STAGE = 128;
-    static constexpr int XBUF = 64 * BN * 4;
-    static constexpr int SWS = 32;               // s_w ring (128 fp32 per step)
-    static constexpr int OFF_ACT = 0;
-    static constexpr int OFF_PK = OFF_ACT + SA * ACT_STAGE;
-    static constexpr int OFF_Z = OFF_PK + SP * PK_STAGE;
-    static constexpr int OFF_SW = OFF_Z + SP * Z_STAGE;
-    static constexpr int OFF_X = OFF_SW + SWS * 512;
-    static constexpr int OFF_BAR = OFF_X + XBUF;
-    static constexpr int NUM_BARS = 2 * SP + 3 * SA + 2 * NACC + 2 * SWS + 1;
-    static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-    static constexpr int BYTES = OFF_MISC + 16;
-    static constexpr int SMEM = BYTES + 1024;    // slack for 1024-byte alignment
-    static constexpr int CH = BN / 2;            // accumulator columns per epilogue thread
+    static constexpr int GW = GROUP / 4;                 // TMEM columns of one unpacked group
+    static constexpr int ACT_TILE = BN * GROUP;          // one group's activation tile
+    static constexpr int PK_HALF = 32 * GROUP;           // one group of one 64-column block
+    // groups per request (chunk) of each stream
+    static constexpr int SGP = GROUP == 128 ? 4 : 8;     // packed codes + zero-points
+    static constexpr int SGA_RAW = 32768 / ACT_TILE;
+    static constexpr int SGA = SGA_RAW < 1 ? 1 : (SGA_RAW > 8 ? 8 : SGA_RAW);  // activation tiles
+    static constexpr int SGW = 8;                        // group scales
+    // ring depths (in chunks) and the TMEM rings (in groups)
+    static constexpr int SPC = (BN == 16) ? 4 : (BN == 128 ? 2 : 3);
+    static constexpr int SAC = (SGA * ACT_TILE <= 16384) ? 3 : (BN == 128 ? 3 : 2);
+    static constexpr int SWC = 4;
+    static constexpr int NACC = BN == 16 ? 8 : BN == 32 ? 8 : BN == 64 ? (GROUP == 128 ? 4 : 6) : 3;
+    static constexpr int SA = BN == 128 && GROUP == 128 ? 4 : 8;
+    static constexpr int A_COL0 = NACC * BN;             // first TMEM column of the A ring
     static constexpr int TMEM_USED = A_COL0 + SA * GW;
     static constexpr uint32_t TMEM_COLS = TMEM_USED <= 32 ? 32 : TMEM_USED <= 64 ? 64 : TMEM_USED <= 128 ? 128
                                           : TMEM_USED <= 256 ? 256 : 512;
+    // shared memory
+    static constexpr int ACT_STAGE = SGA * ACT_TILE;
+    static constexpr int PK_STAGE = 2 * SGP * PK_HALF;   // [half][group][...]
+    static constexpr int Z_STAGE = 2 * SGP * 64;         // [half][group][64 columns]
+    static constexpr int SW_STAGE = 2 * SGW * 64 * 4;    // [half][group][64 columns] fp32
+    static constexpr int XBUF = MODE == kModeGateUp ? 64 * BN * 4 : 0;
+    static constexpr int OFF_ACT = 0;
+    static constexpr int OFF_PK = OFF_ACT + SAC * ACT_STAGE;
+    static constexpr int OFF_Z = OFF_PK + SPC * PK_STAGE;
+    static constexpr int OFF_SW = OFF_Z + SPC * Z_STAGE;
+    static constexpr int OFF_X = OFF_SW + SWC * SW_STAGE;
+    static constexpr int OFF_BAR = OFF_X + XBUF;
+    static constexpr int NUM_BARS = 2 * SPC + 2 * SAC + 2 * SWC + 2 * SA + 2 * NACC + 1;
+    static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+    static constexpr int BYTES = OFF_MISC + 16;
+    static constexpr int SMEM = BYTES + 1024;            // slack for 1024-byte alignment
+    static constexpr int CH = BN / 2;                    // accumulator columns per epilogue thread
     static constexpr uint32_t IDESC = idesc_i8(BN);
     static_assert(BN == 16 || BN == 32 || BN == 64 || BN == 128, "BN");
     static_assert(GROUP == 64 || GROUP == 128, "GROUP");
-    static_assert(ACT_STAGE % 1024 == 0, "swizzle atoms need 1024-byte stages");
-    static_assert(SA >= 2 && SP >= 2 && NACC >= 2, "rings");
+    static_assert(ACT_TILE % 1024 == 0, "swizzle atoms need 1024-byte tiles");
     static_assert(TMEM_USED <= 512, "TMEM columns");
     static_assert(SMEM <= 227 * 1024, "shared memory");
 };
@@ -187,15 +202,40 @@ __device__ __forceinline__ void cta_units(const GemmParams& p, long long& u0, lo
 }
 
 constexpr int kUnpackWarps = 4;
-
 constexpr int kWarpPack = 12, kWarpAct = 13, kWarpMma = 14;
+
+// One tile's run of groups [gb, ge) in this CTA's range.
+struct Segment {
+    long long t;
+    int gb, ge;
+};
+
+__device__ __forceinline__ Segment segment_at(long long u, long long u1, int G) {
+    Segment sg;
+    sg.t = u / G;
+    sg.gb = (int)(u % G);
+    sg.ge = (int)min((long long)G, sg.gb + (u1 - u));
+    return sg;
+}
+
+// Steps back `n` uses of a ring (for the exit drains).
+__device__ __forceinline__ void ring_back(Ring& r, int n) {
+    if (r.idx == 0) {
+        r.idx = n - 1;
+        r.phase ^= 1u;
+    } else {
+        --r.idx;
+    }
+}
 
 // MODE (GemmMode) and DBG (write the int32 group partials) are compile-time,
 // so each launched kernel carries only its own epilogue.
-template <int BN, int GROUP, int SP, int SA, int NACC, int MODE, bool DBG>
+template <int BN, int GROUP, int MODE, bool DBG>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-    w4a8_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act, const GemmParams p) {
-    using C = GemmCfg<BN, GROUP, SP, SA, NACC>;
+    w4a8_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act, const __grid_constant__ CUtensorMap tmap_sw,
+                        const __grid_constant__ CUtensorMap tmap_z, const GemmParams p) {
+    using C = GemmCfg<BN, GROUP, MODE>;
+    constexpr int NACC = C::NACC, SA = C::SA;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sAct = smem + C::OFF_ACT;
@@ -204,16 +244,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     float* sSW = reinterpret_cast<float*>(smem + C::OFF_SW);
     float* sX = reinterpret_cast<float*>(smem + C::OFF_X);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-    uint64_t* p_full = bars;                 // [SP] packed codes (+ z) landed
-    uint64_t* p_empty = p_full + SP;         // [SP] the 4 unpack warps read them
-    uint64_t* act_full = p_empty + SP;       // [SA] activation tile landed
-    uint64_t* a_full = act_full + SA;        // [SA] weight tile unpacked into TMEM
-    uint64_t* a_empty = a_full + SA;         // [SA] MMA done with both
-    uint64_t* acc_full = a_empty + SA;       // [NACC] partial buffer ready
-    uint64_t* acc_empty = acc_full + NACC;   // [NACC] partial buffer drained + re-armed
-    uint64_t* sw_full = acc_empty + NACC;    // [SWS] group scales of the step landed
-    uint64_t* sw_empty = sw_full + C::SWS;   // [SWS] the 8 epilogue warps read them
-    uint64_t* drain = sw_empty + C::SWS;     // [1]
+    uint64_t* p_full = bars;                     // [SPC] packed codes (+ z) of a chunk landed
+    uint64_t* p_empty = p_full + C::SPC;         // [SPC] the 4 unpack warps read them
+    uint64_t* act_full = p_empty + C::SPC;       // [SAC] activation tiles of a chunk landed
+    uint64_t* act_empty = act_full + C::SAC;     // [SAC] MMA done with them
+    uint64_t* sw_full = act_empty + C::SAC;      // [SWC] group scales of a chunk landed
+    uint64_t* sw_empty = sw_full + C::SWC;       // [SWC] the 8 epilogue warps read them
+    uint64_t* a_full = sw_empty + C::SWC;        // [SA] weight tile of a group unpacked into TMEM
+    uint64_t* a_empty = a_full + SA;             // [SA] MMA done with it
+    uint64_t* acc_full = a_empty + SA;           // [NACC] partial buffer ready
+    uint64_t* acc_empty = acc_full + NACC;       // [NACC] partial buffer drained + re-armed
+    uint64_t* drain = acc_empty + NACC;          // [1]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
     int* abort_flag = reinterpret_cast<int*>(smem + C::OFF_MISC + 4);
 
@@ -221,12 +262,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < SP; ++i) {
+        for (int i = 0; i < C::SPC; ++i) {
             mbar_init(&p_full[i], 1);
             mbar_init(&p_empty[i], kUnpackWarps);
         }
-        for (int i = 0; i < SA; ++i) {
+        for (int i = 0; i < C::SAC; ++i) {
             mbar_init(&act_full[i], 1);
+            mbar_init(&act_empty[i], 1);
+        }
+        for (int i = 0; i < C::SWC; ++i) {
+            mbar_init(&sw_full[i], 1);
+            mbar_init(&sw_empty[i], kNumEpiWarps);
+        }
+        for (int i = 0; i < SA; ++i) {
             mbar_init(&a_full[i], kUnpackWarps);
             mbar_init(&a_empty[i], 1);
         }
@@ -234,15 +282,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             mbar_init(&acc_full[i], 1);
             mbar_init(&acc_empty[i], kNumEpiWarps);
         }
-        for (int i = 0; i < C::SWS; ++i) {
-            mbar_init(&sw_full[i], 1);
-            mbar_init(&sw_empty[i], kNumEpiWarps);
-        }
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
         fence_proxy_async_smem();
         prefetch_tmap(&tmap_act);
+        prefetch_tmap(&tmap_sw);
+        if (!p.symmetric) prefetch_tmap(&tmap_z);
     }
     if (warp == kWarpMma) {
         tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -257,104 +303,131 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     long long u0, u1, Q;
     cta_units<MODE>(p, u0, u1, Q);
     const int G = p.G;
-    const long long nsteps = u1 - u0;  // one step = one K-group of one tile
 
-    if (warp == kWarpPack || warp == kWarpAct) {
-        // ------------------------------------------------------ producers --
+    if (warp == kWarpPack) {
+        // ------------------------------------- producer: packed codes (+ z) --
         if (lane == 0) {
-            const bool pack = warp == kWarpPack;
-            const int ring = pack ? SP : SA;
+            Ring rp;
             long long issued = 0;
             bool ok = true;
-            long long t = u0 / G;
-            int gi = (int)(u0 % G);
-            long long cur_t = -1;
-            TileInfo ti{};
-            int nb0 = 0, nb1 = -1;
-            Ring rs, rw;  // this producer's ring; s_w ring (activation producer)
-            for (long long i = 0; i < nsteps; ++i) {
-                if (t != cur_t) {
-                    ti = decode_tile<BN, MODE>(p, t);
-                    tile_blocks<MODE>(p, ti.nt, nb0, nb1);
-                    cur_t = t;
-                }
-                const uint32_t s = rs.idx;
-                if (pack) {
-                    if (!wait_bounded(&p_empty[s], rs.phase ^ 1u, wc)) { ok = false; break; }
-                    uint32_t bytes = C::PK_HALF;
-                    if (nb1 >= 0) bytes += C::PK_HALF;
-                    if (!p.symmetric) bytes += (nb1 >= 0) ? 128 : 64;
-                    mbar_arrive_expect_tx(&p_full[s], bytes);
-                    const uint8_t* wbase = p.packed + (long long)ti.e * p.packed_estride;
-                    uint8_t* pk = sPk + s * C::PK_STAGE;
-                    bulk_load(pk, wbase + ((long long)nb0 * G + gi) * C::PK_HALF, C::PK_HALF, &p_full[s]);
+            for (long long u = u0; u < u1 && ok;) {
+                const Segment sg = segment_at(u, u1, G);
+                const TileInfo ti = decode_tile<BN, MODE>(p, sg.t);
+                int nb0, nb1;
+                tile_blocks<MODE>(p, ti.nt, nb0, nb1);
+                const uint8_t* wbase = p.packed + (long long)ti.e * p.packed_estride;
+                const int zrow = ti.e * G;
+                for (int g0 = sg.gb; g0 < sg.ge; g0 += C::SGP) {
+                    const int clen = min(C::SGP, sg.ge - g0);
+                    if (!wait_bounded(&p_empty[rp.idx], rp.phase ^ 1u, wc)) { ok = false; break; }
+                    const int halves = nb1 >= 0 ? 2 : 1;
+                    uint32_t bytes = halves * clen * C::PK_HALF;
+                    if (!p.symmetric) bytes += halves * C::SGP * 64;
+                    mbar_arrive_expect_tx(&p_full[rp.idx], bytes);
+                    uint8_t* pk = sPk + rp.idx * C::PK_STAGE;
+                    bulk_load(pk, wbase + ((long long)nb0 * G + g0) * C::PK_HALF, clen * C::PK_HALF, &p_full[rp.idx]);
                     if (nb1 >= 0)
-                        bulk_load(pk + C::PK_HALF, wbase + ((long long)nb1 * G + gi) * C::PK_HALF, C::PK_HALF,
-                                  &p_full[s]);
+                        bulk_load(pk + C::SGP * C::PK_HALF, wbase + ((long long)nb1 * G + g0) * C::PK_HALF,
+                                  clen * C::PK_HALF, &p_full[rp.idx]);
                     if (!p.symmetric) {
-                        const uint8_t* zr = p.z + (long long)ti.e * p.sw_estride + (long long)gi * p.N;
-                        bulk_load(sZ + s * C::Z_STAGE, zr + 64 * nb0, 64, &p_full[s]);
-                        if (nb1 >= 0) bulk_load(sZ + s * C::Z_STAGE + 64, zr + 64 * nb1, 64, &p_full[s]);
+                        uint8_t* zs = sZ + rp.idx * C::Z_STAGE;
+                        tma_load_2d(zs, &tmap_z, &p_full[rp.idx], 64 * nb0, zrow + g0);
+                        if (nb1 >= 0) tma_load_2d(zs + C::SGP * 64, &tmap_z, &p_full[rp.idx], 64 * nb1, zrow + g0);
                     }
-                } else {
-                    // group scales of the step's 128 weight rows (read by the epilogue)
-                    const uint32_t w = rw.idx;
-                    if (!wait_bounded(&sw_empty[w], rw.phase ^ 1u, wc)) { ok = false; break; }
-                    mbar_arrive_expect_tx(&sw_full[w], (nb1 >= 0) ? 512 : 256);
-                    const float* swr = p.s_w + (long long)ti.e * p.sw_estride + (long long)gi * p.N;
-                    bulk_load(sSW + w * 128, swr + 64 * nb0, 256, &sw_full[w]);
-                    if (nb1 >= 0) bulk_load(sSW + w * 128 + 64, swr + 64 * nb1, 256, &sw_full[w]);
-                    rw.next(C::SWS);
-                    // activation tile
-                    if (!wait_bounded(&a_empty[s], rs.phase ^ 1u, wc)) { ok = false; break; }
-                    mbar_arrive_expect_tx(&act_full[s], C::ACT_STAGE);
-                    tma_load_2d(sAct + s * C::ACT_STAGE, &tmap_act, &act_full[s], gi * GROUP, ti.row0);
+                    rp.next(C::SPC);
+                    ++issued;
                 }
-                rs.next(ring);
-                ++issued;
-                if (++gi == G) { gi = 0; ++t; }
+                u += sg.ge - sg.gb;
             }
-            (void)ok;
-            // Drain: wait for the last issue of every stage, so no copy is in
-            // flight into shared memory when the CTA exits.
+            // Drain: the last copy of every stage lands before the CTA exits.
             WaitCtx wd{abort_flag, p.status, wait_cycles_for_ns(p.wait_ns)};
             volatile int no_abort = 0;
-            wd.abort = &no_abort;  // drain even after an abort
-            uint64_t* fullb = pack ? p_full : act_full;
-            Ring d = rs;
-            for (long long k = 0; k < issued && k < ring; ++k) {
-                if (d.idx == 0) { d.idx = ring - 1; d.phase ^= 1u; } else { --d.idx; }
-                (void)wait_bounded(&fullb[d.idx], d.phase, wd);
+            wd.abort = &no_abort;
+            Ring d = rp;
+            for (long long k = 0; k < issued && k < C::SPC; ++k) {
+                ring_back(d, C::SPC);
+                (void)wait_bounded(&p_full[d.idx], d.phase, wd);
             }
-            if (!pack) {
-                const long long nsw = issued + (ok ? 0 : 1);  // an s_w copy may precede a failed wait
-                Ring dw = rw;
-                for (long long k = 0; k < nsw && k < C::SWS; ++k) {
-                    if (dw.idx == 0) { dw.idx = C::SWS - 1; dw.phase ^= 1u; } else { --dw.idx; }
-                    (void)wait_bounded(&sw_full[dw.idx], dw.phase, wd);
+        }
+    } else if (warp == kWarpAct) {
+        // ------------------------- producer: activation tiles, group scales --
+        if (lane == 0) {
+            Ring ra, rw;
+            long long na = 0, nw = 0;
+            bool ok = true;
+            for (long long u = u0; u < u1 && ok;) {
+                const Segment sg = segment_at(u, u1, G);
+                const TileInfo ti = decode_tile<BN, MODE>(p, sg.t);
+                int nb0, nb1;
+                tile_blocks<MODE>(p, ti.nt, nb0, nb1);
+                const int wrow = ti.e * G;
+                for (int g = sg.gb; g < sg.ge; ++g) {
+                    const int j = g - sg.gb;
+                    if (j % C::SGW == 0) {
+                        if (!wait_bounded(&sw_empty[rw.idx], rw.phase ^ 1u, wc)) { ok = false; break; }
+                        mbar_arrive_expect_tx(&sw_full[rw.idx], (nb1 >= 0 ? 2 : 1) * C::SGW * 256);
+                        float* ws = sSW + rw.idx * (C::SW_STAGE / 4);
+                        tma_load_2d(ws, &tmap_sw, &sw_full[rw.idx], 64 * nb0, wrow + g);
+                        if (nb1 >= 0) tma_load_2d(ws + C::SGW * 64, &tmap_sw, &sw_full[rw.idx], 64 * nb1, wrow + g);
+                        rw.next(C::SWC);
+                        ++nw;
+                    }
+                    if (j % C::SGA == 0) {
+                        if (!wait_bounded(&act_empty[ra.idx], ra.phase ^ 1u, wc)) { ok = false; break; }
+                        mbar_arrive_expect_tx(&act_full[ra.idx], C::ACT_STAGE);
+                        tma_load_3d(sAct + ra.idx * C::ACT_STAGE, &tmap_act, &act_full[ra.idx], 0, ti.row0, g);
+                        ra.next(C::SAC);
+                        ++na;
+                    }
                 }
+                u += sg.ge - sg.gb;
+            }
+            WaitCtx wd{abort_flag, p.status, wait_cycles_for_ns(p.wait_ns)};
+            volatile int no_abort = 0;
+            wd.abort = &no_abort;
+            Ring d = ra;
+            for (long long k = 0; k < na && k < C::SAC; ++k) {
+                ring_back(d, C::SAC);
+                (void)wait_bounded(&act_full[d.idx], d.phase, wd);
+            }
+            Ring dw = rw;
+            for (long long k = 0; k < nw && k < C::SWC; ++k) {
+                ring_back(dw, C::SWC);
+                (void)wait_bounded(&sw_full[dw.idx], dw.phase, wd);
             }
         }
     } else if (warp == kWarpMma) {
         // ----------------------------------------------------- MMA issue --
         if (lane == 0) {
             const uint32_t b_base = smem_u32(sAct);
-            Ring ra, rc;
-            for (long long i = 0; i < nsteps; ++i, ra.next(SA), rc.next(NACC)) {
-                const uint32_t sa = ra.idx;
-                const uint32_t ab = rc.idx;
-                if (!wait_bounded(&act_full[sa], ra.phase, wc)) break;
-                if (!wait_bounded(&a_full[sa], ra.phase, wc)) break;
-                if (!wait_bounded(&acc_empty[ab], rc.phase, wc)) break;
-                tc_fence_after();
-                const uint64_t bdesc = umma_desc_kmajor(b_base + sa * C::ACT_STAGE, GROUP);
-                const uint32_t a_tmem = tmem_base + C::A_COL0 + sa * C::GW;
-                const uint32_t d_tmem = tmem_base + ab * BN;
+            Ring ra, rt, rc;
+            bool ok = true;
+            for (long long u = u0; u < u1 && ok;) {
+                const Segment sg = segment_at(u, u1, G);
+                for (int g = sg.gb; g < sg.ge; ++g) {
+                    const int j = (g - sg.gb) % C::SGA;
+                    const int cend = min(C::SGA, sg.ge - (g - j)) - 1;
+                    if (j == 0 && !wait_bounded(&act_full[ra.idx], ra.phase, wc)) { ok = false; break; }
+                    if (!wait_bounded(&a_full[rt.idx], rt.phase, wc)) { ok = false; break; }
+                    if (!wait_bounded(&acc_empty[rc.idx], rc.phase, wc)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint64_t bdesc =
+                        umma_desc_kmajor(b_base + ra.idx * C::ACT_STAGE + j * C::ACT_TILE, GROUP);
+                    const uint32_t a_tmem = tmem_base + C::A_COL0 + rt.idx * C::GW;
+                    const uint32_t d_tmem = tmem_base + rc.idx * BN;
 #pragma unroll
-                for (int kk = 0; kk < GROUP / 32; ++kk)
-                    mma_i8_tmem_a(d_tmem, a_tmem + 8 * kk, bdesc + 2 * kk, C::IDESC, 1u);
-                tc_commit(&a_empty[sa]);
-                tc_commit(&acc_full[ab]);
+                    for (int kk = 0; kk < GROUP / 32; ++kk)
+                        mma_i8_tmem_a(d_tmem, a_tmem + 8 * kk, bdesc + 2 * kk, C::IDESC, 1u);
+                    tc_commit(&a_empty[rt.idx]);
+                    tc_commit(&acc_full[rc.idx]);
+                    if (j == cend) {
+                        tc_commit(&act_empty[ra.idx]);
+                        ra.next(C::SAC);
+                    }
+                    rt.next(SA);
+                    rc.next(NACC);
+                }
+                u += sg.ge - sg.gb;
             }
             // Drain: every MMA issued above completes before TMEM is freed.
             tc_commit(drain);
@@ -365,7 +438,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
     } else if (warp < kUnpackWarps) {
         // ---------------------------------------------------------- unpack --
-        // Warp q turns rows 32q..32q+31 of every step's weight tile into int8
+        // Warp q turns rows 32q..32q+31 of every group's weight tile into int8
         // and stores them in TMEM lanes 32q..32q+31 (row = lane).
         const int r = warp * 32 + lane;
         const int half = r >> 6, rr = r & 63;
@@ -373,52 +446,55 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // Each byte: 0x80 | code (sym: code ^ 8 = q + 8), minus z (sym: 8),
         // then ^ 0x80: the two's complement int8 of (q - z) in [-15, 15].
         const uint32_t k1 = p.symmetric ? 0x88888888u : 0x80808080u;
-        long long cur_t = -1;
-        int nb1 = -1;
-        long long t = u0 / G;
-        int gi = (int)(u0 % G);
         Ring rp, ra;
-        for (long long i = 0; i < nsteps; ++i, rp.next(SP), ra.next(SA)) {
-            if (t != cur_t) {
-                const TileInfo ti = decode_tile<BN, MODE>(p, t);
-                int nb0;
-                tile_blocks<MODE>(p, ti.nt, nb0, nb1);
-                cur_t = t;
-            }
-            if (++gi == G) { gi = 0; ++t; }
+        bool ok = true;
+        for (long long u = u0; u < u1 && ok;) {
+            const Segment sg = segment_at(u, u1, G);
+            const TileInfo ti = decode_tile<BN, MODE>(p, sg.t);
+            int nb0, nb1;
+            tile_blocks<MODE>(p, ti.nt, nb0, nb1);
             const bool row_valid = (half == 0) || (nb1 >= 0);
-            const uint32_t ps = rp.idx;
-            if (!warp_wait_bounded(&p_full[ps], rp.phase, wc)) break;
-            uint4 w[GROUP / 32];
-            uint32_t zz = 0x08080808u;
-            const uint8_t* pk = sPk + ps * C::PK_STAGE + half * C::PK_HALF;
+            for (int g = sg.gb; g < sg.ge; ++g) {
+                const int j = (g - sg.gb) % C::SGP;
+                const int cend = min(C::SGP, sg.ge - (g - j)) - 1;
+                if (j == 0 && !warp_wait_bounded(&p_full[rp.idx], rp.phase, wc)) { ok = false; break; }
+                uint4 w[GROUP / 32];
+                uint32_t zz = 0x08080808u;
+                const uint8_t* pk = sPk + rp.idx * C::PK_STAGE + (half * C::SGP + j) * C::PK_HALF;
 #pragma unroll
-            for (int c = 0; c < GROUP / 32; ++c)
-                w[c] = row_valid ? *reinterpret_cast<const uint4*>(pk + (c * 64 + rr) * 16) : make_uint4(0, 0, 0, 0);
-            if (!p.symmetric) zz = 0x01010101u * (uint32_t)sZ[ps * C::Z_STAGE + r];
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&p_empty[ps]);
-            // TMEM column 8c + j holds k = 32c + 4j .. 32c + 4j + 3
-            uint32_t out[C::GW];
-#pragma unroll
-            for (int c = 0; c < GROUP / 32; ++c) {
-                const uint32_t ws[4] = {w[c].x, w[c].y, w[c].z, w[c].w};
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const uint32_t lo = (((ws[j] & 0x0F0F0F0Fu) ^ k1) - zz) ^ 0x80808080u;
-                    const uint32_t hi = ((((ws[j] >> 4) & 0x0F0F0F0Fu) ^ k1) - zz) ^ 0x80808080u;
-                    out[8 * c + j] = row_valid ? lo : 0u;
-                    out[8 * c + 4 + j] = row_valid ? hi : 0u;
+                for (int c = 0; c < GROUP / 32; ++c)
+                    w[c] = row_valid ? *reinterpret_cast<const uint4*>(pk + (c * 64 + rr) * 16)
+                                     : make_uint4(0, 0, 0, 0);
+                if (!p.symmetric)
+                    zz = 0x01010101u * (uint32_t)sZ[rp.idx * C::Z_STAGE + (half * C::SGP + j) * 64 + rr];
+                if (j == cend) {
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&p_empty[rp.idx]);
+                    rp.next(C::SPC);
                 }
+                // TMEM column 8c + i holds k = 32c + 4i .. 32c + 4i + 3
+                uint32_t out[C::GW];
+#pragma unroll
+                for (int c = 0; c < GROUP / 32; ++c) {
+                    const uint32_t ws[4] = {w[c].x, w[c].y, w[c].z, w[c].w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const uint32_t lo = (((ws[i] & 0x0F0F0F0Fu) ^ k1) - zz) ^ 0x80808080u;
+                        const uint32_t hi = ((((ws[i] >> 4) & 0x0F0F0F0Fu) ^ k1) - zz) ^ 0x80808080u;
+                        out[8 * c + i] = row_valid ? lo : 0u;
+                        out[8 * c + 4 + i] = row_valid ? hi : 0u;
+                    }
+                }
+                if (!warp_wait_bounded(&a_empty[ra.idx], ra.phase ^ 1u, wc)) { ok = false; break; }
+                tc_fence_after();
+                tmem_st32<C::GW>(tmem_base + lane_addr + C::A_COL0 + ra.idx * C::GW, out);
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&a_full[ra.idx]);
+                ra.next(SA);
             }
-            const uint32_t sa = ra.idx;
-            if (!warp_wait_bounded(&a_empty[sa], ra.phase ^ 1u, wc)) break;
-            tc_fence_after();
-            tmem_st32<C::GW>(tmem_base + lane_addr + C::A_COL0 + sa * C::GW, out);
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&a_full[sa]);
+            u += sg.ge - sg.gb;
         }
     } else if (warp < kUnpackWarps + kNumEpiWarps) {
         // -------------------------------------------------------- epilogue --
@@ -426,6 +502,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int q = warp & 3;              // TMEM lane quadrant this warp may access
         const int hcol = ew >> 2;            // column half
         const int r = q * 32 + lane;         // weight row within the tile
+        const int half = r >> 6;
         constexpr int CH = C::CH;
         const uint32_t lane_addr = ((uint32_t)(q * 32)) << 16;
 
@@ -449,13 +526,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         bool ok = true;
         Ring rw, rc;
         for (long long u = u0; u < u1 && ok;) {
-            const long long t = u / G;
-            const int gb = (int)(u % G);
-            const int ge = (int)min((long long)G, gb + (u1 - u));
+            const Segment sg = segment_at(u, u1, G);
+            const long long t = sg.t;
+            const int gb = sg.gb, ge = sg.ge;
             const TileInfo ti = decode_tile<BN, MODE>(p, t);
             int nb0, nb1;
             tile_blocks<MODE>(p, ti.nt, nb0, nb1);
-            const int half = r >> 6;
             const bool n_valid = (half == 0) || (nb1 >= 0);
             const int n = (half == 0 ? nb0 : nb1) * 64 + (r & 63);  // weight column
 
@@ -463,12 +539,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
             for (int jj = 0; jj < CH; ++jj) acc[jj] = 0.0f;
 
-            for (int gi = gb; gi < ge; ++gi, rw.next(C::SWS), rc.next(NACC)) {
-                const uint32_t w = rw.idx;
-                if (!warp_wait_bounded(&sw_full[w], rw.phase, wc)) { ok = false; break; }
-                const float sw = n_valid ? sSW[w * 128 + r] : 0.0f;
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sw_empty[w]);
+            for (int gi = gb; gi < ge; ++gi) {
+                const int j = (gi - gb) % C::SGW;
+                const int cend = min(C::SGW, ge - (gi - j)) - 1;
+                if (j == 0 && !warp_wait_bounded(&sw_full[rw.idx], rw.phase, wc)) { ok = false; break; }
+                const float sw = n_valid ? sSW[rw.idx * (C::SW_STAGE / 4) + (half * C::SGW + j) * 64 + (r & 63)]
+                                         : 0.0f;
+                if (j == cend) {
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sw_empty[rw.idx]);
+                    rw.next(C::SWC);
+                }
                 const uint32_t ab = rc.idx;
                 if (!warp_wait_bounded(&acc_full[ab], rc.phase, wc)) { ok = false; break; }
                 tc_fence_after();
@@ -498,6 +579,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&acc_empty[ab]);
+                rc.next(NACC);
             }
             if constexpr (MODE == kModeGateUp) {
                 // The exchange below uses named barriers: decide together

@@ -55,20 +55,49 @@ EncodeTiledFn get_encode_fn() {
     return fn;
 }
 
-// Tensor map over an int8 [rows][K] row-major matrix, box = group x bn,
-// swizzle = group bytes (64B or 128B).
-bool make_act_tmap(CUtensorMap* map, const void* base, int rows, int K, int group, int bn) {
+// Tensor map over the int8 activations [rows][K] seen as 3-D
+// (k within group, row, group), box = group x bn x (groups per request);
+// swizzle = group bytes (64B or 128B), matching the MMA's K-major layout.
+bool make_act_tmap(CUtensorMap* map, const void* base, int rows, int K, int group, int bn, int chunk) {
     EncodeTiledFn enc = get_encode_fn();
     if (!enc) return false;
-    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)K};
-    cuuint32_t box[2] = {(cuuint32_t)group, (cuuint32_t)bn};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+    cuuint64_t dims[3] = {(cuuint64_t)group, (cuuint64_t)rows, (cuuint64_t)(K / group)};
+    cuuint64_t strides[2] = {(cuuint64_t)K, (cuuint64_t)group};
+    cuuint32_t box[3] = {(cuuint32_t)group, (cuuint32_t)bn, (cuuint32_t)chunk};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE,
                      group == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
+}
+
+// Tensor map over a [rows][N] matrix (fp32 scales or uint8 zero-points),
+// box = 64 columns x `chunk` rows.
+bool make_cols_tmap(CUtensorMap* map, const void* base, long long rows, int N, bool f32, int chunk) {
+    EncodeTiledFn enc = get_encode_fn();
+    if (!enc) return false;
+    const int es = f32 ? 4 : 1;
+    cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)N * es};
+    cuuint32_t box[2] = {64, (cuuint32_t)chunk};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+                     const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// All three maps of one GEMM launch.
+bool make_gemm_maps(GemmMaps* m, const void* act, int rows, int K, int group, int bn, int mode, const float* s_w,
+                    const uint8_t* z, int E, int N) {
+    std::memset(m, 0, sizeof(*m));
+    const long long wrows = (long long)E * (K / group);
+    if (!make_act_tmap(&m->act, act, rows, K, group, bn, chunk_act(bn, group, mode))) return false;
+    if (!make_cols_tmap(&m->sw, s_w, wrows, N, true, kChunkScales)) return false;
+    if (z && !make_cols_tmap(&m->z, z, wrows, N, false, chunk_packed(group))) return false;
+    return true;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -78,14 +107,14 @@ w4a8_status last_cuda() { return cudaGetLastError() == cudaSuccess ? W4A8_OK : W
 // ---------------------------------------------------------- GEMM configs --
 
 // GEMM launch: per-mode entry points live in gemm_<mode>.cu (see gemm_launch.cuh).
-w4a8_status launch_gemm(int mode, bool dbg, int bn, int group, const CUtensorMap& tmap, const GemmParams& p,
+w4a8_status launch_gemm(int mode, bool dbg, int bn, int group, const GemmMaps& maps, const GemmParams& p,
                         int grid, cudaStream_t stream) {
     int r;
     switch (mode) {
-        case kModePlain: r = launch_gemm_plain(dbg, bn, group, tmap, p, grid, stream); break;
-        case kModeSplitK: r = launch_gemm_splitk(dbg, bn, group, tmap, p, grid, stream); break;
-        case kModeGateUp: r = launch_gemm_gateup(bn, group, tmap, p, grid, stream); break;
-        case kModeDown: r = launch_gemm_down(bn, group, tmap, p, grid, stream); break;
+        case kModePlain: r = launch_gemm_plain(dbg, bn, group, maps, p, grid, stream); break;
+        case kModeSplitK: r = launch_gemm_splitk(dbg, bn, group, maps, p, grid, stream); break;
+        case kModeGateUp: r = launch_gemm_gateup(bn, group, maps, p, grid, stream); break;
+        case kModeDown: r = launch_gemm_down(bn, group, maps, p, grid, stream); break;
         default: r = W4A8_ERR_UNSUPPORTED_SHAPE;
     }
     return static_cast<w4a8_status>(r);
@@ -155,8 +184,9 @@ w4a8_status gemm_impl(const int8_t* qx, const float* s_x, const uint8_t* packed,
     const GemmPlan pl = plan_gemm(M, w->N, w->K, w->group, sm_count_current());
     if (pl.ws_bytes > 0 && (!workspace || ws_bytes < pl.ws_bytes)) return W4A8_ERR_WORKSPACE;
 
-    CUtensorMap tmap;
-    if (!make_act_tmap(&tmap, qx, M, w->K, w->group, pl.bn)) return W4A8_ERR_CUDA;
+    const int mode = pl.splitk ? kModeSplitK : kModePlain;
+    GemmMaps maps;
+    if (!make_gemm_maps(&maps, qx, M, w->K, w->group, pl.bn, mode, s_w, z, 1, w->N)) return W4A8_ERR_CUDA;
     GemmParams p{};
     p.packed = packed;
     p.s_w = s_w;
@@ -179,7 +209,7 @@ w4a8_status gemm_impl(const int8_t* qx, const float* s_x, const uint8_t* packed,
     p.status = dev_status;
     p.wait_ns = kDefaultWaitNs;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    st = launch_gemm(p.mode, P != nullptr, pl.bn, w->group, tmap, p, pl.grid, s);
+    st = launch_gemm(p.mode, P != nullptr, pl.bn, w->group, maps, p, pl.grid, s);
     if (st != W4A8_OK) return st;
     if (pl.splitk) {
         const long long n = (long long)M * w->N;
@@ -426,8 +456,8 @@ w4a8_status w4a8_moe_grouped_gemm_profiled(const uint16_t* X, const float* logit
     // 4. gate_up + SiLU * up
     if (!mark(3)) return W4A8_ERR_CUDA;
     {
-        CUtensorMap tmap;
-        if (!make_act_tmap(&tmap, qx, R, H, group, bn)) return W4A8_ERR_CUDA;
+        GemmMaps maps;
+        if (!make_gemm_maps(&maps, qx, R, H, group, bn, kModeGateUp, w1_s, w1_z, E, w1->N)) return W4A8_ERR_CUDA;
         GemmParams p{};
         p.packed = w1_packed;
         p.s_w = w1_s;
@@ -449,7 +479,7 @@ w4a8_status w4a8_moe_grouped_gemm_profiled(const uint16_t* X, const float* logit
         p.I = I;
         p.status = dev_status;
         p.wait_ns = kDefaultWaitNs;
-        if ((st = launch_gemm(kModeGateUp, false, bn, group, tmap, p, sms, s)) != W4A8_OK) return st;
+        if ((st = launch_gemm(kModeGateUp, false, bn, group, maps, p, sms, s)) != W4A8_OK) return st;
     }
     // 5. quantize h per (token, expert) row
     if (!mark(4)) return W4A8_ERR_CUDA;
@@ -457,8 +487,8 @@ w4a8_status w4a8_moe_grouped_gemm_profiled(const uint16_t* X, const float* logit
     // 6. down
     if (!mark(5)) return W4A8_ERR_CUDA;
     {
-        CUtensorMap tmap;
-        if (!make_act_tmap(&tmap, qh, R, I, group, bn)) return W4A8_ERR_CUDA;
+        GemmMaps maps;
+        if (!make_gemm_maps(&maps, qh, R, I, group, bn, kModeDown, w2_s, w2_z, E, H)) return W4A8_ERR_CUDA;
         GemmParams p{};
         p.packed = w2_packed;
         p.s_w = w2_s;
@@ -479,7 +509,7 @@ w4a8_status w4a8_moe_grouped_gemm_profiled(const uint16_t* X, const float* logit
         p.E = E;
         p.status = dev_status;
         p.wait_ns = kDefaultWaitNs;
-        if ((st = launch_gemm(kModeDown, false, bn, group, tmap, p, sms, s)) != W4A8_OK) return st;
+        if ((st = launch_gemm(kModeDown, false, bn, group, maps, p, sms, s)) != W4A8_OK) return st;
     }
     // 7. weighted combine
     if (!mark(6)) return W4A8_ERR_CUDA;
