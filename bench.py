@@ -507,16 +507,40 @@ def run_ours(args, world, rank, local):
         dist.destroy_process_group()
 
 
+def kernel_sources_sha256():
+    """Digest of the kernel sources; a stored ncu traffic figure is only used
+    while the sources it was measured on are unchanged."""
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "moe_linear_layers_w4a8_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            h.update(name.encode())
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(f.read())
+    return h.hexdigest()
+
+
 def traffic_from_profiles(workload, roof):
     """DRAM bytes per launch of the dominant kernel from the committed ncu
-    summary (profiles/*.json), or None when no current capture exists."""
-    path = os.path.join(ROOT, "profiles", "traffic.json")
+    summary profiles/traffic.txt, or None when it was taken on other sources."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
     try:
         with open(path) as f:
-            d = json.load(f)
-        return d.get(workload)
-    except Exception:
+            lines = f.read().splitlines()
+    except OSError:
         return None
+    sha, table = None, {}
+    for ln in lines:
+        if ln.startswith("# sources-sha256:"):
+            sha = ln.split(":", 1)[1].strip()
+        elif ln and not ln.startswith("#"):
+            parts = ln.split()
+            if len(parts) >= 2:
+                table[parts[0]] = int(parts[1])
+    if sha != kernel_sources_sha256():
+        return None
+    return table.get(workload)
 
 
 def cpu_baseline(wl, unit_scale, unit, budget_s=12.0):
