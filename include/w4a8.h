@@ -191,6 +191,44 @@ W4A8_API w4a8_status w4a8_gemm_debug_partials(const int8_t* qx, const float* s_x
                                      int32_t* dev_status, void* stream);
 
 /*
+ * w4a8_gemm_static_scratch — w4a8_gemm for callers that cannot allocate.
+ * The pages have no counterpart of this call: it is a library-integration
+ * entry point, not a step of the method.  It computes exactly what w4a8_gemm
+ * computes, with the same kernels.
+ *
+ * Who needs it: callers with no device allocator at the call site, or that
+ * must not use one there — a plain C host that links libw4a8.so without a
+ * framework and owns no scratch buffer; code running while a caching
+ * allocator's pool is capped or frozen; decode loops where cudaMalloc /
+ * cudaFree would synchronize the device or can fail under memory pressure.
+ * Instead of the caller's workspace, the split-K partials go to one fixed
+ * buffer of W4A8_STATIC_SCRATCH_BYTES per device, compiled into the library
+ * (a static __device__ array).  This call allocates and frees nothing.
+ *
+ * Set-up: the first call on each device looks up the buffer's device address
+ * with that device current (cudaGetSymbolAddress; this may load the
+ * library's device code).  Make that first call before any stream capture.
+ * Sharing: every call on a device uses the same buffer.  Two calls whose
+ * kernels can overlap on the GPU (different streams without an ordering
+ * between them, or concurrent host threads) race on it and give wrong
+ * results: issue them on one stream or order them.
+ * Nothing in the buffer has to start at zero: each call writes every partial
+ * it later reads.
+ * Limit: a call whose plan needs more than W4A8_STATIC_SCRATCH_BYTES (i.e.
+ * w4a8_gemm_workspace_size(M, w) > W4A8_STATIC_SCRATCH_BYTES; for instance
+ * M = 64 with K = 4096, N = 14336) returns W4A8_ERR_WORKSPACE and launches
+ * nothing; use w4a8_gemm with a workspace then.  Shapes that need no scratch
+ * (large M) run as in w4a8_gemm.
+ * Arguments and other errors: as w4a8_gemm, without workspace / ws_bytes;
+ * W4A8_ERR_CUDA if the address lookup fails.
+ */
+#define W4A8_STATIC_SCRATCH_BYTES ((size_t)8 << 20)
+W4A8_API w4a8_status w4a8_gemm_static_scratch(const int8_t* qx, const float* s_x,
+                                     const uint8_t* packed, const float* s_w, const uint8_t* z,
+                                     const w4a8_wdesc* w, int M, uint16_t* Y, int ldy,
+                                     int32_t* dev_status, void* stream);
+
+/*
  * w4a8_moe_grouped_gemm — one MoE expert layer, following "Kimi 2.7 MoE,
  * 4-bit storage to INT8" §4.1-4.4:
  *   1. routing in fp32 (the router stays in high precision): topk_idx = the

@@ -19,7 +19,7 @@ import torch
 __all__ = [
     "W4A8Error", "WDesc", "PackedWeight", "load_library", "library_path",
     "w4a8_pack_weights", "w4a8_pack_expert_weights", "w4a8_quant_act", "w4a8_gemm",
-    "w4a8_gemm_debug_partials", "w4a8_moe_grouped_gemm", "w4a8_moe_workspace_layout",
+    "w4a8_gemm_debug_partials", "w4a8_gemm_static_scratch", "w4a8_moe_grouped_gemm", "w4a8_moe_workspace_layout",
     "w4a8_gemm_workspace_size", "w4a8_moe_workspace_size", "w4a8_get_device_status",
     "w4a8_status_string", "w4a8_selftest_bounded_wait", "w4a8_linear", "LAYOUT_VERSION",
     "STATUS",
@@ -108,6 +108,8 @@ def load_library():
         L.w4a8_quant_act.argtypes = [P, I, I, I, I, P, P, P, P, P]
         L.w4a8_gemm.restype = st
         L.w4a8_gemm.argtypes = [P, P, P, P, P, ctypes.POINTER(WDesc), I, P, I, P, S, P, P]
+        L.w4a8_gemm_static_scratch.restype = st
+        L.w4a8_gemm_static_scratch.argtypes = [P, P, P, P, P, ctypes.POINTER(WDesc), I, P, I, P, P]
         L.w4a8_gemm_debug_partials.restype = st
         L.w4a8_gemm_debug_partials.argtypes = [P, P, P, P, P, ctypes.POINTER(WDesc), I, P, I, P, P, S, P, P]
         L.w4a8_moe_grouped_gemm.restype = st
@@ -256,6 +258,21 @@ def w4a8_gemm(qx: torch.Tensor, s_x: torch.Tensor, w: PackedWeight, out: Optiona
               workspace: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None) -> torch.Tensor:
     """Y bf16 [M, N] = W4A8(qx, w)."""
     return _gemm(qx, s_x, w, out, workspace, status, None)
+
+
+def w4a8_gemm_static_scratch(qx: torch.Tensor, s_x: torch.Tensor, w: PackedWeight, out: torch.Tensor,
+                             status: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """w4a8_gemm without a workspace: the library's fixed per-device scratch
+    buffer holds the split-K partials, and nothing is allocated (``out`` is
+    required).  Calls that may overlap on the GPU race on that buffer."""
+    L = load_library()
+    _need_cuda(qx, s_x)
+    if qx.dtype != torch.int8 or qx.dim() != 2 or not qx.is_contiguous():
+        raise W4A8Error(1, "qx must be contiguous int8 [M, K]")
+    code = L.w4a8_gemm_static_scratch(_p(qx), _p(s_x), _p(w.packed), _p(w.s_w), _p(w.z), ctypes.byref(w.desc),
+                                      qx.shape[0], _p(out), out.stride(0), _p(status), _stream(qx.device))
+    _check(code, "w4a8_gemm_static_scratch")
+    return out
 
 
 def w4a8_gemm_debug_partials(qx, s_x, w: PackedWeight, out=None, workspace=None, status=None):

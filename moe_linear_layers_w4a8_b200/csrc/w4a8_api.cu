@@ -549,3 +549,51 @@ w4a8_status w4a8_selftest_bounded_wait(int32_t* dev_status, uint64_t limit_ns, v
 }
 
 }  // extern "C"
+
+// ------------------------------------------------ static-scratch GEMM entry --
+//
+// w4a8_gemm_static_scratch: w4a8_gemm for callers that cannot allocate (see
+// include/w4a8.h).  The split-K partials live in the fixed buffer below
+// instead of a caller workspace.  `g_static_scratch` names the buffer on the
+// host side only; it is not a device address.  The device address comes from
+// cudaGetSymbolAddress, looked up once per device with that device current.
+
+namespace {
+
+static __device__ __align__(256) unsigned char g_static_scratch[W4A8_STATIC_SCRATCH_BYTES];
+
+constexpr int kMaxScratchDevices = 64;
+std::mutex g_scratch_mutex;
+void* g_scratch_ptr[kMaxScratchDevices] = {};
+
+// Device address of g_static_scratch on the current device, or null.
+void* static_scratch_current_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxScratchDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(g_scratch_mutex);
+    if (!g_scratch_ptr[dev]) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_static_scratch) != cudaSuccess) return nullptr;
+        g_scratch_ptr[dev] = ptr;
+    }
+    return g_scratch_ptr[dev];
+}
+
+}  // namespace
+
+extern "C" w4a8_status w4a8_gemm_static_scratch(const int8_t* qx, const float* s_x, const uint8_t* packed,
+                                                const float* s_w, const uint8_t* z, const w4a8_wdesc* w, int M,
+                                                uint16_t* Y, int ldy, int32_t* dev_status, void* stream) {
+    w4a8_status st = check_wdesc(w);
+    if (st != W4A8_OK) return st;
+    if (M < 0) return W4A8_ERR_INVALID_ARG;
+    const size_t need = M > 0 ? plan_gemm(M, w->N, w->K, w->group, sm_count_current()).ws_bytes : 0;
+    if (need > W4A8_STATIC_SCRATCH_BYTES) return W4A8_ERR_WORKSPACE;
+    void* scratch = nullptr;
+    if (need > 0) {
+        scratch = static_scratch_current_device();
+        if (!scratch) return W4A8_ERR_CUDA;
+    }
+    return gemm_impl(qx, s_x, packed, s_w, z, w, M, Y, ldy, nullptr, scratch, need > 0 ? W4A8_STATIC_SCRATCH_BYTES : 0,
+                     dev_status, stream);
+}
