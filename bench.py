@@ -398,13 +398,19 @@ def barrier_sync(torch, world):
     torch.cuda.synchronize()
 
 
-def max_over_ranks(torch, world, v):
+def max_over_ranks(torch, world, v, device="cuda"):
+    """The slowest rank's time: every rank gets the max (one all-reduce)."""
     if world == 1:
         return v
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(unit_scale, steps, world, t_ms):
+    """Whole-job rate: the units all ranks processed over the slowest rank's time."""
+    return unit_scale * steps * world / (t_ms / 1e3)
 
 
 def run_ours(args, world, rank, local):
@@ -444,7 +450,7 @@ def run_ours(args, world, rank, local):
     t_ms = start.elapsed_time(end)
     t_ms = max_over_ranks(torch, world, t_ms)
     ms_per_step = t_ms / K
-    value = unit_scale * K * world / (t_ms / 1e3)
+    value = job_throughput(unit_scale, K, world, t_ms)
 
     # dominant-kernel time: events around its launches in the last replay
     stage_ms = None
@@ -479,7 +485,7 @@ def run_ours(args, world, rank, local):
     e2.record()
     torch.cuda.synchronize()
     te = max_over_ranks(torch, world, s2.elapsed_time(e2))
-    e2e_value = unit_scale * Ke * world / (te / 1e3)
+    e2e_value = job_throughput(unit_scale, Ke, world, te)
 
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": unit, "n_gpus": world, "steps": K, "warmup": W,
