@@ -17,26 +17,37 @@
 //   * The unpacked int8 weight tile lives in TMEM (tcgen05.mma with A from
 //     TMEM): each unpack thread turns one row of packed codes into int8 in
 //     registers and writes the whole row of the group with one tcgen05.st,
-//     so the only shared-memory traffic per step is the packed codes and the
+//     so the only shared-memory traffic per group is the packed codes and the
 //     activation tile.
 //   * Warp roles (512 threads): warps 0-3 unpack (warp q owns TMEM lanes /
 //     weight rows 32q..32q+31), warps 4-11 drain the partial sums, warp 12
-//     brings packed codes (TMA bulk copies, deep ring), warp 13 brings
-//     activation tiles (tiled TMA), one lane of warp 14 issues the MMAs.
-//   * TMEM holds NACC int32 partial buffers.  Each is pre-filled with
-//     0x4B400000 before a group's MMAs, so afterwards it holds the bits of
-//     the float 12582912 + P (|P| < 2^22): one FADD turns it into P exactly,
-//     one FFMA applies s_w.
-//   * K is walked one quantization group per MMA step, but every TMA request
-//     brings several consecutive groups ("chunks"): the packed codes of up to
-//     4 (g=128) / 8 (g=64) groups per 64-column half, the activation tiles of
-//     up to 8 groups through a 3-D tensor map (k within group, row, group),
-//     and the scales / zero-points of 8 groups through 2-D tensor maps.  An
-//     SM's TMA unit spends a roughly fixed time per request, so few large
-//     requests keep it off the critical path.
+//     brings packed codes (TMA bulk copies), warp 13 brings activation tiles
+//     (tiled TMA) and scales, one lane of warp 14 issues the MMAs.
+//   * The pipeline advances in steps of S consecutive K-groups of one tile
+//     (S = 4 for BN <= 32, 2 for 64, 1 for 128).  A step owns one TMEM
+//     "slot": S unpacked weight tiles and S int32 partial buffers.  Three
+//     barriers per slot-use and one MMA commit per step: the MMA thread waits
+//     once (`ready`: all 4 unpack warps wrote the weight tiles and all 8
+//     epilogue warps drained the buffers' previous use), issues S x GROUP/32
+//     MMAs and commits once (`done`: weight tiles free, partials ready).
+//     Every fixed per-step cost (barrier waits, commits, fences) is paid once
+//     per S groups.
+//   * Each partial buffer is pre-filled with 0x4B400000 before its MMAs, so
+//     afterwards it holds the bits of the float 12582912 + P (|P| < 2^22):
+//     one FADD turns it into P exactly, one FFMA applies s_w.
+//   * Every TMA request brings several consecutive groups ("chunks"): the
+//     packed codes of up to 4 (g=128) / 8 (g=64) groups per 64-column half,
+//     the activation tiles of up to 8 groups through a 3-D tensor map (k
+//     within group, row, group), and the scales / zero-points of 8 groups
+//     through 2-D tensor maps.
 //   * Persistent: each CTA owns a contiguous range of (tile, group) units.
-//     Ranges that split a tile (split-K) write fp32 partial tiles that a
-//     second kernel sums in a fixed order.
+//     When ranges split a tile (split-K), the CTA holding the tile's first
+//     groups sums it: the other contributors (later CTAs, whose ranges start
+//     inside the tile) store fp32 partial tiles plus a flag set to the
+//     launch's epoch; the summing CTA waits (bounded) for those flags, clears
+//     them, adds the partials in slot order and writes the output.  It only
+//     waits on CTAs with higher indices, which never wait on it, so no cycle
+//     of waits exists; a flag left by another launch holds another epoch.
 //   * Every mbarrier wait is bounded; on expiry the CTA records
 //     W4A8_ERR_TIMEOUT, drains its in-flight copies and MMAs, frees TMEM and
 //     exits.
@@ -64,8 +75,10 @@ struct GemmParams {
     int mode;
     uint16_t* Y;                 // plain: Y; gate_up: h; down: expert outputs
     int ldy;
-    float* partial;              // split-K partial tiles
+    float* partial;              // split-K partial tiles [tiles][slots][BN][128]
     int slots;                   // split-K slots per tile
+    unsigned long long* flags;   // split-K: [tiles][slots] "partial stored" flags (epoch values)
+    unsigned long long epoch;    // this launch's epoch (nonzero)
     int32_t* dbgP;               // optional [M][G][N] int32 partials (plain / split-K)
     int n_tiles;
     int m_tiles;                 // plain / split-K
@@ -76,6 +89,7 @@ struct GemmParams {
     int I;                       // gate_up: intermediate size
     int32_t* status;
     unsigned long long wait_ns;
+    int vec16;                   // Y and ldy allow 16-byte row stores
 };
 
 constexpr int kGemmThreads = 512;  // 4 unpack, 8 epilogue, 2 producer, 1 MMA, 1 spare warp
@@ -94,14 +108,17 @@ struct GemmCfg {
     static constexpr int SGA_RAW = 32768 / ACT_TILE;
     static constexpr int SGA = SGA_RAW < 1 ? 1 : (SGA_RAW > 8 ? 8 : SGA_RAW);  // activation tiles
     static constexpr int SGW = 8;                        // group scales
-    // ring depths (in chunks) and the TMEM rings (in groups)
+    // pipeline steps: S groups per step, NS TMEM slots of S (weight tile + partial buffer)
+    static constexpr int S = BN <= 32 ? 4 : (BN == 64 ? 2 : 1);
+    static constexpr int SLOT_COLS = S * (GW + BN);
+    static constexpr int NS_RAW = 512 / SLOT_COLS;
+    static constexpr int NS = NS_RAW > 4 ? 4 : NS_RAW;
+    // ring depths of the shared-memory streams (in chunks)
     static constexpr int SPC = (BN == 16) ? 4 : (BN == 128 ? 2 : 3);
     static constexpr int SAC = (SGA * ACT_TILE <= 16384) ? 3 : (BN == 128 ? 3 : 2);
     static constexpr int SWC = 4;
-    static constexpr int NACC = BN == 16 ? 8 : BN == 32 ? 8 : BN == 64 ? (GROUP == 128 ? 4 : 6) : 3;
-    static constexpr int SA = BN == 128 && GROUP == 128 ? 4 : 8;
-    static constexpr int A_COL0 = NACC * BN;             // first TMEM column of the A ring
-    static constexpr int TMEM_USED = A_COL0 + SA * GW;
+    static constexpr int A_COL0 = NS * S * BN;           // first TMEM column of the weight tiles
+    static constexpr int TMEM_USED = NS * SLOT_COLS;
     static constexpr uint32_t TMEM_COLS = TMEM_USED <= 32 ? 32 : TMEM_USED <= 64 ? 64 : TMEM_USED <= 128 ? 128
                                           : TMEM_USED <= 256 ? 256 : 512;
     // shared memory
@@ -110,13 +127,15 @@ struct GemmCfg {
     static constexpr int Z_STAGE = 2 * SGP * 64;         // [half][group][64 columns]
     static constexpr int SW_STAGE = 2 * SGW * 64 * 4;    // [half][group][64 columns] fp32
     static constexpr int XBUF = MODE == kModeGateUp ? 64 * BN * 4 : 0;
+    static constexpr int YBUF = MODE == kModeGateUp ? 0 : BN * 128 * 2;   // bf16 output tile staging
     static constexpr int OFF_ACT = 0;
     static constexpr int OFF_PK = OFF_ACT + SAC * ACT_STAGE;
     static constexpr int OFF_Z = OFF_PK + SPC * PK_STAGE;
     static constexpr int OFF_SW = OFF_Z + SPC * Z_STAGE;
     static constexpr int OFF_X = OFF_SW + SWC * SW_STAGE;
-    static constexpr int OFF_BAR = OFF_X + XBUF;
-    static constexpr int NUM_BARS = 2 * SPC + 2 * SAC + 2 * SWC + 2 * SA + 2 * NACC + 1;
+    static constexpr int OFF_Y = OFF_X + XBUF;
+    static constexpr int OFF_BAR = OFF_Y + YBUF;
+    static constexpr int NUM_BARS = 2 * SPC + 2 * SAC + 2 * SWC + 2 * NS + 1;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
     static constexpr int BYTES = OFF_MISC + 16;
     static constexpr int SMEM = BYTES + 1024;            // slack for 1024-byte alignment
@@ -125,7 +144,8 @@ struct GemmCfg {
     static_assert(BN == 16 || BN == 32 || BN == 64 || BN == 128, "BN");
     static_assert(GROUP == 64 || GROUP == 128, "GROUP");
     static_assert(ACT_TILE % 1024 == 0, "swizzle atoms need 1024-byte tiles");
-    static_assert(TMEM_USED <= 512, "TMEM columns");
+    static_assert(SGP % S == 0 && SGA % S == 0 && SGW % S == 0, "a step never straddles a chunk");
+    static_assert(NS >= 1 && TMEM_USED <= 512, "TMEM columns");
     static_assert(SMEM <= 227 * 1024, "shared memory");
 };
 
@@ -228,6 +248,41 @@ __device__ __forceinline__ void ring_back(Ring& r, int n) {
     }
 }
 
+// s_x of the tile's activation rows col0 .. col0 + JW - 1, all loads issued
+// back to back (indices clamped into the tile's valid rows; the values of
+// clamped columns are never stored).
+template <int JW>
+__device__ __forceinline__ void load_sx(const float* s_x, const TileInfo& ti, int col0, float* sx) {
+#pragma unroll
+    for (int jj = 0; jj < JW; ++jj) sx[jj] = __ldg(s_x + ti.row0 + min(col0 + jj, ti.rows_valid - 1));
+}
+
+// Copies a bf16 output tile staged in shared memory ([BN rows][128 columns])
+// to Y: 16-byte row segments, one per thread and iteration (256 epilogue
+// threads), skipping rows past the tile's valid rows and columns past ncols.
+template <int BN>
+__device__ __forceinline__ void store_staged_tile(const uint16_t* sY, const GemmParams& p, const TileInfo& ti,
+                                                  int n0, int ncols, int et) {
+#pragma unroll
+    for (int c = et; c < BN * 16; c += kNumEpiWarps * 32) {
+        const int row = c >> 4, seg = c & 15;
+        if (row < ti.rows_valid && seg * 8 < ncols) {
+            const uint4 v = *reinterpret_cast<const uint4*>(sY + row * 128 + seg * 8);
+            uint16_t* dst = p.Y + (long long)(ti.row0 + row) * p.ldy + n0 + seg * 8;
+            if (p.vec16) {
+                *reinterpret_cast<uint4*>(dst) = v;
+            } else {
+                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    dst[2 * k] = (uint16_t)(w[k] & 0xFFFFu);
+                    dst[2 * k + 1] = (uint16_t)(w[k] >> 16);
+                }
+            }
+        }
+    }
+}
+
 // MODE (GemmMode) and DBG (write the int32 group partials) are compile-time,
 // so each launched kernel carries only its own epilogue.
 template <int BN, int GROUP, int MODE, bool DBG>
@@ -235,7 +290,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     w4a8_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act, const __grid_constant__ CUtensorMap tmap_sw,
                         const __grid_constant__ CUtensorMap tmap_z, const GemmParams p) {
     using C = GemmCfg<BN, GROUP, MODE>;
-    constexpr int NACC = C::NACC, SA = C::SA;
+    constexpr int S = C::S, NS = C::NS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sAct = smem + C::OFF_ACT;
@@ -243,6 +298,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint8_t* sZ = smem + C::OFF_Z;
     float* sSW = reinterpret_cast<float*>(smem + C::OFF_SW);
     float* sX = reinterpret_cast<float*>(smem + C::OFF_X);
+    uint16_t* sY = reinterpret_cast<uint16_t*>(smem + C::OFF_Y);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
     uint64_t* p_full = bars;                     // [SPC] packed codes (+ z) of a chunk landed
     uint64_t* p_empty = p_full + C::SPC;         // [SPC] the 4 unpack warps read them
@@ -250,11 +306,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint64_t* act_empty = act_full + C::SAC;     // [SAC] MMA done with them
     uint64_t* sw_full = act_empty + C::SAC;      // [SWC] group scales of a chunk landed
     uint64_t* sw_empty = sw_full + C::SWC;       // [SWC] the 8 epilogue warps read them
-    uint64_t* a_full = sw_empty + C::SWC;        // [SA] weight tile of a group unpacked into TMEM
-    uint64_t* a_empty = a_full + SA;             // [SA] MMA done with it
-    uint64_t* acc_full = a_empty + SA;           // [NACC] partial buffer ready
-    uint64_t* acc_empty = acc_full + NACC;       // [NACC] partial buffer drained + re-armed
-    uint64_t* drain = acc_empty + NACC;          // [1]
+    uint64_t* ready = sw_empty + C::SWC;         // [NS] slot's weight tiles written + partial buffers re-armed
+    uint64_t* done = ready + NS;                 // [NS] slot's MMAs complete
+    uint64_t* drain = done + NS;                 // [1]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
     int* abort_flag = reinterpret_cast<int*>(smem + C::OFF_MISC + 4);
 
@@ -274,13 +328,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             mbar_init(&sw_full[i], 1);
             mbar_init(&sw_empty[i], kNumEpiWarps);
         }
-        for (int i = 0; i < SA; ++i) {
-            mbar_init(&a_full[i], kUnpackWarps);
-            mbar_init(&a_empty[i], 1);
-        }
-        for (int i = 0; i < NACC; ++i) {
-            mbar_init(&acc_full[i], 1);
-            mbar_init(&acc_empty[i], kNumEpiWarps);
+        for (int i = 0; i < NS; ++i) {
+            mbar_init(&ready[i], kUnpackWarps + kNumEpiWarps);
+            mbar_init(&done[i], 1);
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -400,32 +450,36 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // ----------------------------------------------------- MMA issue --
         if (lane == 0) {
             const uint32_t b_base = smem_u32(sAct);
-            Ring ra, rt, rc;
+            Ring ra, rs;
             bool ok = true;
             for (long long u = u0; u < u1 && ok;) {
                 const Segment sg = segment_at(u, u1, G);
-                for (int g = sg.gb; g < sg.ge; ++g) {
-                    const int j = (g - sg.gb) % C::SGA;
-                    const int cend = min(C::SGA, sg.ge - (g - j)) - 1;
+                for (int g0 = sg.gb; g0 < sg.ge; g0 += S) {
+                    const int ns = min(S, sg.ge - g0);
+                    const int j = (g0 - sg.gb) % C::SGA;            // position in the activation chunk
+                    const int clen = min(C::SGA, sg.ge - (g0 - j));  // groups in that chunk
                     if (j == 0 && !wait_bounded(&act_full[ra.idx], ra.phase, wc)) { ok = false; break; }
-                    if (!wait_bounded(&a_full[rt.idx], rt.phase, wc)) { ok = false; break; }
-                    if (!wait_bounded(&acc_empty[rc.idx], rc.phase, wc)) { ok = false; break; }
+                    if (!wait_bounded(&ready[rs.idx], rs.phase, wc)) { ok = false; break; }
                     tc_fence_after();
-                    const uint64_t bdesc =
-                        umma_desc_kmajor(b_base + ra.idx * C::ACT_STAGE + j * C::ACT_TILE, GROUP);
-                    const uint32_t a_tmem = tmem_base + C::A_COL0 + rt.idx * C::GW;
-                    const uint32_t d_tmem = tmem_base + rc.idx * BN;
+                    const uint32_t b0 = b_base + ra.idx * C::ACT_STAGE + j * C::ACT_TILE;
+                    const uint32_t slot0 = rs.idx * S;
 #pragma unroll
-                    for (int kk = 0; kk < GROUP / 32; ++kk)
-                        mma_i8_tmem_a(d_tmem, a_tmem + 8 * kk, bdesc + 2 * kk, C::IDESC, 1u);
-                    tc_commit(&a_empty[rt.idx]);
-                    tc_commit(&acc_full[rc.idx]);
-                    if (j == cend) {
+                    for (int i = 0; i < S; ++i) {
+                        if (i < ns) {
+                            const uint64_t bdesc = umma_desc_kmajor(b0 + i * C::ACT_TILE, GROUP);
+                            const uint32_t a_tmem = tmem_base + C::A_COL0 + (slot0 + i) * C::GW;
+                            const uint32_t d_tmem = tmem_base + (slot0 + i) * BN;
+#pragma unroll
+                            for (int kk = 0; kk < GROUP / 32; ++kk)
+                                mma_i8_tmem_a(d_tmem, a_tmem + 8 * kk, bdesc + 2 * kk, C::IDESC, 1u);
+                        }
+                    }
+                    tc_commit(&done[rs.idx]);
+                    if (j + ns == clen) {
                         tc_commit(&act_empty[ra.idx]);
                         ra.next(C::SAC);
                     }
-                    rt.next(SA);
-                    rc.next(NACC);
+                    rs.next(NS);
                 }
                 u += sg.ge - sg.gb;
             }
@@ -439,60 +493,82 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     } else if (warp < kUnpackWarps) {
         // ---------------------------------------------------------- unpack --
         // Warp q turns rows 32q..32q+31 of every group's weight tile into int8
-        // and stores them in TMEM lanes 32q..32q+31 (row = lane).
+        // and stores them in TMEM lanes 32q..32q+31 (row = lane).  Rows of an
+        // absent 64-column half are unpacked from whatever the stage holds:
+        // their partials are never read.
         const int r = warp * 32 + lane;
         const int half = r >> 6, rr = r & 63;
         const uint32_t lane_addr = ((uint32_t)(warp * 32)) << 16;
-        // Each byte: 0x80 | code (sym: code ^ 8 = q + 8), minus z (sym: 8),
-        // then ^ 0x80: the two's complement int8 of (q - z) in [-15, 15].
-        const uint32_t k1 = p.symmetric ? 0x88888888u : 0x80808080u;
-        Ring rp, ra;
+        Ring rp, rs;
         bool ok = true;
         for (long long u = u0; u < u1 && ok;) {
             const Segment sg = segment_at(u, u1, G);
-            const TileInfo ti = decode_tile<BN, MODE>(p, sg.t);
-            int nb0, nb1;
-            tile_blocks<MODE>(p, ti.nt, nb0, nb1);
-            const bool row_valid = (half == 0) || (nb1 >= 0);
-            for (int g = sg.gb; g < sg.ge; ++g) {
-                const int j = (g - sg.gb) % C::SGP;
-                const int cend = min(C::SGP, sg.ge - (g - j)) - 1;
-                if (j == 0 && !warp_wait_bounded(&p_full[rp.idx], rp.phase, wc)) { ok = false; break; }
-                uint4 w[GROUP / 32];
-                uint32_t zz = 0x08080808u;
-                const uint8_t* pk = sPk + rp.idx * C::PK_STAGE + (half * C::SGP + j) * C::PK_HALF;
+            for (int g0 = sg.gb; g0 < sg.ge; g0 += S) {
+                const int ns = min(S, sg.ge - g0);
+                const int jp = (g0 - sg.gb) % C::SGP;             // position in the packed chunk
+                const int plen = min(C::SGP, sg.ge - (g0 - jp));  // groups in that chunk
+                if (jp == 0 && !warp_wait_bounded(&p_full[rp.idx], rp.phase, wc)) { ok = false; break; }
+                // the slot's weight tiles are free once its previous MMAs completed
+                if (!warp_wait_bounded(&done[rs.idx], rs.phase ^ 1u, wc)) { ok = false; break; }
+                tc_fence_after();
+                const uint8_t* pk = sPk + rp.idx * C::PK_STAGE + (half * C::SGP + jp) * C::PK_HALF + rr * 16;
+                const uint8_t* zp = sZ + rp.idx * C::Z_STAGE + (half * C::SGP + jp) * 64 + rr;
+                const uint32_t a0 = tmem_base + lane_addr + C::A_COL0 + rs.idx * S * C::GW;
+                // packed words of group i + 1 are loaded while group i is unpacked
+                uint4 wb[2][GROUP / 32];
 #pragma unroll
-                for (int c = 0; c < GROUP / 32; ++c)
-                    w[c] = row_valid ? *reinterpret_cast<const uint4*>(pk + (c * 64 + rr) * 16)
-                                     : make_uint4(0, 0, 0, 0);
-                if (!p.symmetric)
-                    zz = 0x01010101u * (uint32_t)sZ[rp.idx * C::Z_STAGE + (half * C::SGP + j) * 64 + rr];
-                if (j == cend) {
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&p_empty[rp.idx]);
-                    rp.next(C::SPC);
-                }
-                // TMEM column 8c + i holds k = 32c + 4i .. 32c + 4i + 3
-                uint32_t out[C::GW];
+                for (int c = 0; c < GROUP / 32; ++c) wb[0][c] = *reinterpret_cast<const uint4*>(pk + c * 1024);
 #pragma unroll
-                for (int c = 0; c < GROUP / 32; ++c) {
-                    const uint32_t ws[4] = {w[c].x, w[c].y, w[c].z, w[c].w};
+                for (int i = 0; i < S; ++i) {
+                    if (i < ns) {
+                        if (i + 1 < ns) {
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const uint32_t lo = (((ws[i] & 0x0F0F0F0Fu) ^ k1) - zz) ^ 0x80808080u;
-                        const uint32_t hi = ((((ws[i] >> 4) & 0x0F0F0F0Fu) ^ k1) - zz) ^ 0x80808080u;
-                        out[8 * c + i] = row_valid ? lo : 0u;
-                        out[8 * c + 4 + i] = row_valid ? hi : 0u;
+                            for (int c = 0; c < GROUP / 32; ++c)
+                                wb[(i + 1) & 1][c] =
+                                    *reinterpret_cast<const uint4*>(pk + (i + 1) * C::PK_HALF + c * 1024);
+                        }
+                        // TMEM column 8c + q holds k = 32c + 4q .. 32c + 4q + 3
+                        uint32_t out[C::GW];
+                        if (p.symmetric) {
+                            // A 4-bit two's complement code moved to the top of
+                            // its byte is the int8 16 q: the tile holds 16 q_w
+                            // and the MMA yields 16 P exactly (|16 P| < 2^21).
+#pragma unroll
+                            for (int c = 0; c < GROUP / 32; ++c) {
+                                const uint4 w = wb[i & 1][c];
+                                const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                                for (int q = 0; q < 4; ++q) {
+                                    out[8 * c + q] = (ws[q] << 4) & 0xF0F0F0F0u;
+                                    out[8 * c + 4 + q] = ws[q] & 0xF0F0F0F0u;
+                                }
+                            }
+                        } else {
+                            // Each byte: 0x80 | u, minus z, then ^ 0x80: the int8 u - z.
+                            const uint32_t zz = 0x01010101u * (uint32_t)zp[i * 64];
+#pragma unroll
+                            for (int c = 0; c < GROUP / 32; ++c) {
+                                const uint4 w = wb[i & 1][c];
+                                const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                                for (int q = 0; q < 4; ++q) {
+                                    out[8 * c + q] = (((ws[q] & 0x0F0F0F0Fu) | 0x80808080u) - zz) ^ 0x80808080u;
+                                    out[8 * c + 4 + q] = ((((ws[q] >> 4) & 0x0F0F0F0Fu) | 0x80808080u) - zz) ^ 0x80808080u;
+                                }
+                            }
+                        }
+                        tmem_st32<C::GW>(a0 + i * C::GW, out);
                     }
                 }
-                if (!warp_wait_bounded(&a_empty[ra.idx], ra.phase ^ 1u, wc)) { ok = false; break; }
-                tc_fence_after();
-                tmem_st32<C::GW>(tmem_base + lane_addr + C::A_COL0 + ra.idx * C::GW, out);
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&a_full[ra.idx]);
-                ra.next(SA);
+                if (lane == 0) {
+                    if (jp + ns == plen) mbar_arrive(&p_empty[rp.idx]);
+                    mbar_arrive(&ready[rs.idx]);
+                }
+                if (jp + ns == plen) rp.next(C::SPC);
+                rs.next(NS);
             }
             u += sg.ge - sg.gb;
         }
@@ -504,28 +580,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int r = q * 32 + lane;         // weight row within the tile
         const int half = r >> 6;
         constexpr int CH = C::CH;
+        // A step's partials are read in batches of BC columns (all groups of
+        // the step when they fit in 32 registers), one TMEM wait per batch.
+        constexpr int LDW = CH < 16 ? CH : 16;                              // columns per tcgen05.ld
+        constexpr int BC = CH >= 64 ? 16 : (S * CH < 32 ? S * CH : 32);    // columns per batch (register budget)
+        constexpr int NBAT = S * CH / BC;
+        static_assert(BC % LDW == 0 && (BC % CH == 0 || CH % BC == 0), "batches");
         const uint32_t lane_addr = ((uint32_t)(q * 32)) << 16;
 
-        // Arm every partial buffer, then hand them to the MMA warp.
+        // Arm every partial buffer of every slot, then release the slots.
 #pragma unroll
-        for (int b = 0; b < NACC; ++b) {
+        for (int b = 0; b < NS * S; ++b) {
             const uint32_t ta = tmem_base + lane_addr + b * BN + hcol * CH;
-            if constexpr (CH >= 32) {
 #pragma unroll
-                for (int c0 = 0; c0 < CH; c0 += 32) tmem_fill32<32>(ta + c0, kMagicBits);
-            } else {
-                tmem_fill32<CH>(ta, kMagicBits);
-            }
+            for (int c0 = 0; c0 < CH; c0 += LDW) tmem_fill32<LDW>(ta + c0, kMagicBits);
         }
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0)
-            for (int b = 0; b < NACC; ++b) mbar_arrive(&acc_empty[b]);
+            for (int b = 0; b < NS; ++b) mbar_arrive(&ready[b]);
 
         bool ok = true;
-        Ring rw, rc;
-        for (long long u = u0; u < u1 && ok;) {
+        Ring rw, rs;
+        for (long long u = u0; u < u1;) {
             const Segment sg = segment_at(u, u1, G);
             const long long t = sg.t;
             const int gb = sg.gb, ge = sg.ge;
@@ -535,42 +613,73 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const bool n_valid = (half == 0) || (nb1 >= 0);
             const int n = (half == 0 ? nb0 : nb1) * 64 + (r & 63);  // weight column
 
-            float acc[CH];
+            // fp32 sums of the group partials, as pairs of adjacent columns
+            uint64_t acc2[CH / 2];
 #pragma unroll
-            for (int jj = 0; jj < CH; ++jj) acc[jj] = 0.0f;
+            for (int jj = 0; jj < CH / 2; ++jj) acc2[jj] = 0ull;
+            const uint64_t neg_magic = f2_splat(-kMagicF);
+            const float psc = p.symmetric ? 0.0625f : 1.0f;
+            const int pshift = p.symmetric ? 4 : 0;
 
-            for (int gi = gb; gi < ge; ++gi) {
-                const int j = (gi - gb) % C::SGW;
-                const int cend = min(C::SGW, ge - (gi - j)) - 1;
-                if (j == 0 && !warp_wait_bounded(&sw_full[rw.idx], rw.phase, wc)) { ok = false; break; }
-                const float sw = n_valid ? sSW[rw.idx * (C::SW_STAGE / 4) + (half * C::SGW + j) * 64 + (r & 63)]
-                                         : 0.0f;
-                if (j == cend) {
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&sw_empty[rw.idx]);
-                    rw.next(C::SWC);
+            for (int g0 = gb; g0 < ge && ok; g0 += S) {
+                const int ns = min(S, ge - g0);
+                // scales of the step's groups
+                uint64_t sw2[S];
+#pragma unroll
+                for (int i = 0; i < S; ++i) {
+                    sw2[i] = 0ull;
+                    if (i < ns) {
+                        const int gi = g0 + i;
+                        const int jw = (gi - gb) % C::SGW;
+                        const int wlen = min(C::SGW, ge - (gi - jw));
+                        if (jw == 0 && !warp_wait_bounded(&sw_full[rw.idx], rw.phase, wc)) { ok = false; break; }
+                        // symmetric tiles hold 16 P: s_w / 16 is exact, so s_w/16 * 16P rounds like s_w * P
+                        sw2[i] = f2_splat(
+                            n_valid ? sSW[rw.idx * (C::SW_STAGE / 4) + (half * C::SGW + jw) * 64 + (r & 63)] * psc
+                                    : 0.0f);
+                        if (jw == wlen - 1) {
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(&sw_empty[rw.idx]);
+                            rw.next(C::SWC);
+                        }
+                    }
                 }
-                const uint32_t ab = rc.idx;
-                if (!warp_wait_bounded(&acc_full[ab], rc.phase, wc)) { ok = false; break; }
+                if (!ok) break;
+                if (!warp_wait_bounded(&done[rs.idx], rs.phase, wc)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t ta = tmem_base + lane_addr + ab * BN + hcol * CH;
-                constexpr int CW = CH < 16 ? CH : 16;  // columns per TMEM load
+                const uint32_t tslot = tmem_base + lane_addr + rs.idx * S * BN + hcol * CH;
+                const int last_b = (ns * CH + BC - 1) / BC - 1;  // last batch holding groups of this step
 #pragma unroll
-                for (int c0 = 0; c0 < CH; c0 += CW) {
-                    uint32_t v[CW];
-                    tmem_ld32<CW>(ta + c0, v);
-                    tmem_wait_ld();
-                    tmem_fill32<CW>(ta + c0, kMagicBits);  // re-arm for the next group
+                for (int b = 0; b < NBAT; ++b) {
+                    if (b <= last_b) {
+                        uint32_t v[BC];
 #pragma unroll
-                    for (int jj = 0; jj < CW; ++jj)
-                        acc[c0 + jj] = fmaf(sw, __uint_as_float(v[jj]) - kMagicF, acc[c0 + jj]);
-                    if (DBG && n_valid) {
+                        for (int x = 0; x < BC; x += LDW) {
+                            const int f = b * BC + x, i = f / CH, c = f % CH;
+                            if (i < ns) tmem_ld32<LDW>(tslot + i * BN + c, v + x);
+                        }
+                        tmem_wait_ld();
 #pragma unroll
-                        for (int jj = 0; jj < CW; ++jj) {
-                            const int col = hcol * CH + c0 + jj;
-                            if (col < ti.rows_valid) {
-                                const long long m = ti.row0 + col;
-                                p.dbgP[(m * G + gi) * p.N + n] = (int32_t)(v[jj] - kMagicBits);
+                        for (int x = 0; x < BC; x += LDW) {  // re-arm for the slot's next use
+                            const int f = b * BC + x, i = f / CH, c = f % CH;
+                            if (i < ns) tmem_fill32<LDW>(tslot + i * BN + c, kMagicBits);
+                        }
+#pragma unroll
+                        for (int x = 0; x < BC; x += 2) {
+                            const int f = b * BC + x, i = f / CH, c = f % CH;
+                            // (12582912 + P) - 12582912 = P exactly; acc += s_w P
+                            if (i < ns)
+                                acc2[c / 2] = f2_fma(sw2[i], f2_add(f2_from_bits(v[x], v[x + 1]), neg_magic), acc2[c / 2]);
+                        }
+                        if (DBG && n_valid) {
+#pragma unroll
+                            for (int x = 0; x < BC; ++x) {
+                                const int f = b * BC + x, i = f / CH, c = f % CH;
+                                const int col = hcol * CH + c;
+                                if (i < ns && col < ti.rows_valid) {
+                                    const long long m = ti.row0 + col;
+                                    p.dbgP[(m * G + g0 + i) * p.N + n] = ((int32_t)(v[x] - kMagicBits)) >> pshift;
+                                }
                             }
                         }
                     }
@@ -578,62 +687,140 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&acc_empty[ab]);
-                rc.next(NACC);
+                if (lane == 0) mbar_arrive(&ready[rs.idx]);
+                rs.next(NS);
             }
-            if constexpr (MODE == kModeGateUp) {
-                // The exchange below uses named barriers: decide together
-                // whether any epilogue warp gave up, so none waits alone.
-                if (named_bar_or(2, kNumEpiWarps * 32, !ok)) break;
-            } else if (!ok) {
-                break;
-            }
+            float acc[CH];
+#pragma unroll
+            for (int jj = 0; jj < CH / 2; ++jj) f2_split(acc2[jj], acc[2 * jj], acc[2 * jj + 1]);
+            // The output below uses named barriers: decide together whether
+            // any epilogue warp gave up, so none waits alone.
+            if (named_bar_or(2, kNumEpiWarps * 32, !ok)) break;
+            const int et = ew * 32 + lane;  // 0..255
+            const int n0 = nb0 * 64, ncols = nb1 >= 0 ? 128 : 64;
 
             // ---------------------------------------------- tile output --
-            const bool full_tile = (gb == 0 && ge == G);
             if constexpr (MODE == kModeSplitK) {
-                const long long c_first = (t * G) / Q;
-                const long long slot = (long long)blockIdx.x - c_first;
-                float* dst = p.partial + ((t * p.slots + slot) * BN) * 128 + r;
+                const bool full_tile = (gb == 0 && ge == G);
+                if (full_tile) {
+                    named_bar_sync(4, kNumEpiWarps * 32);  // the previous tile's copy-out is done with sY
+                    constexpr int JW = CH < 16 ? CH : 16;
 #pragma unroll
-                for (int jj = 0; jj < CH; ++jj) dst[(long long)(hcol * CH + jj) * 128] = acc[jj];
+                    for (int j0 = 0; j0 < CH; j0 += JW) {
+                        float sx[JW];
+                        load_sx<JW>(p.s_x, ti, hcol * CH + j0, sx);
+#pragma unroll
+                        for (int jj = 0; jj < JW; ++jj)
+                            sY[(hcol * CH + j0 + jj) * 128 + r] = f32_to_bf16_bits(sx[jj] * acc[j0 + jj]);
+                    }
+                    named_bar_sync(4, kNumEpiWarps * 32);
+                    store_staged_tile<BN>(sY, p, ti, n0, ncols, et);
+                } else {
+                    // Split tile.  The CTA holding the tile's first groups
+                    // (slot 0) sums it; every other contributor stores its
+                    // fp32 partial tile and then its flag (the launch's epoch).
+                    // A contributor's range starts inside the tile, so its
+                    // partial is stored early in its run, while slot 0 reaches
+                    // the tile at the end of its own run.
+                    const long long c_first = (t * G) / Q;
+                    const int nsl = (int)((t * G + G - 1) / Q - c_first) + 1;
+                    const int slot = (int)((long long)blockIdx.x - c_first);
+                    float* tile_part = p.partial + (t * p.slots) * (BN * 128);
+                    unsigned long long* flags = p.flags + t * p.slots;
+                    if (slot != 0) {
+                        float* dst = tile_part + (long long)slot * (BN * 128) + r;
+#pragma unroll
+                        for (int jj = 0; jj < CH; ++jj) dst[(hcol * CH + jj) * 128] = acc[jj];
+                        __threadfence();
+                        named_bar_sync(3, kNumEpiWarps * 32);
+                        if (ew == 0 && lane == 0) st_release_gpu_u64(flags + slot, p.epoch);
+                    } else {
+                        if (ew == 0) {
+                            bool got = true;
+                            if (lane >= 1 && lane < nsl) {
+                                got = spin_until_equal_u64(flags + lane, p.epoch, wc);
+                                if (got) st_release_gpu_u64(flags + lane, 0ull);  // consumed
+                            }
+                            if (!__all_sync(0xFFFFFFFFu, got) && lane == 0) *wc.abort = 1;
+                        }
+                        named_bar_sync(3, kNumEpiWarps * 32);
+                        const bool reduce = !*wc.abort;
+                        if (reduce) {
+                            __threadfence();
+                            // slot order: own partial first, then slots 1, 2, ...
+                            constexpr int JW = CH < 16 ? CH : 16;
+#pragma unroll
+                            for (int j0 = 0; j0 < CH; j0 += JW) {
+                                float tot[JW];
+#pragma unroll
+                                for (int jj = 0; jj < JW; ++jj) tot[jj] = acc[j0 + jj];
+                                for (int c = 1; c < nsl; ++c) {
+                                    const float* src =
+                                        tile_part + (long long)c * (BN * 128) + (hcol * CH + j0) * 128 + r;
+                                    float v[JW];
+#pragma unroll
+                                    for (int jj = 0; jj < JW; ++jj) v[jj] = __ldcg(src + jj * 128);
+#pragma unroll
+                                    for (int jj = 0; jj < JW; ++jj) tot[jj] += v[jj];
+                                }
+                                float sx[JW];
+                                load_sx<JW>(p.s_x, ti, hcol * CH + j0, sx);
+#pragma unroll
+                                for (int jj = 0; jj < JW; ++jj)
+                                    sY[(hcol * CH + j0 + jj) * 128 + r] = f32_to_bf16_bits(sx[jj] * tot[jj]);
+                            }
+                        }
+                        named_bar_sync(4, kNumEpiWarps * 32);
+                        if (reduce) store_staged_tile<BN>(sY, p, ti, n0, ncols, et);
+                        named_bar_sync(4, kNumEpiWarps * 32);  // sY is free again
+                    }
+                }
             } else if constexpr (MODE == kModeGateUp) {
                 // rows 64..127 hold "up", rows 0..63 the matching "gate"
+                constexpr int JW = CH < 16 ? CH : 16;
                 if (half == 1) {
 #pragma unroll
-                    for (int jj = 0; jj < CH; ++jj) {
-                        const int col = hcol * CH + jj;
-                        const float sx = (col < ti.rows_valid) ? __ldg(p.s_x + ti.row0 + col) : 0.0f;
-                        sX[col * 64 + (r - 64)] = sx * acc[jj];
+                    for (int j0 = 0; j0 < CH; j0 += JW) {
+                        float sx[JW];
+                        load_sx<JW>(p.s_x, ti, hcol * CH + j0, sx);
+#pragma unroll
+                        for (int jj = 0; jj < JW; ++jj) sX[(hcol * CH + j0 + jj) * 64 + (r - 64)] = sx[jj] * acc[j0 + jj];
                     }
                 }
                 named_bar_sync(1, kNumEpiWarps * 32);
                 if (half == 0) {
                     const int ii = ti.nt * 64 + r;
 #pragma unroll
-                    for (int jj = 0; jj < CH; ++jj) {
-                        const int col = hcol * CH + jj;
-                        if (col < ti.rows_valid) {
-                            const long long m = ti.row0 + col;
-                            const float gte = __ldg(p.s_x + m) * acc[jj];
-                            const float up = sX[col * 64 + r];
-                            const float hv = (gte / (1.0f + expf(-gte))) * up;
-                            p.Y[m * p.ldy + ii] = f32_to_bf16_bits(hv);
+                    for (int j0 = 0; j0 < CH; j0 += JW) {
+                        float sx[JW];
+                        load_sx<JW>(p.s_x, ti, hcol * CH + j0, sx);
+#pragma unroll
+                        for (int jj = 0; jj < JW; ++jj) {
+                            const int col = hcol * CH + j0 + jj;
+                            if (col < ti.rows_valid) {
+                                const float gte = sx[jj] * acc[j0 + jj];
+                                const float up = sX[col * 64 + r];
+                                const float hv = (gte / (1.0f + expf(-gte))) * up;
+                                p.Y[(long long)(ti.row0 + col) * p.ldy + ii] = f32_to_bf16_bits(hv);
+                            }
                         }
                     }
                 }
                 named_bar_sync(1, kNumEpiWarps * 32);
             } else {
-                if (full_tile && n_valid) {
+                // plain / down: every range holds whole tiles
+                named_bar_sync(4, kNumEpiWarps * 32);  // the previous tile's copy-out is done with sY
+                constexpr int JW = CH < 16 ? CH : 16;
 #pragma unroll
-                    for (int jj = 0; jj < CH; ++jj) {
-                        const int col = hcol * CH + jj;
-                        if (col < ti.rows_valid) {
-                            const long long m = ti.row0 + col;
-                            p.Y[m * p.ldy + n] = f32_to_bf16_bits(__ldg(p.s_x + m) * acc[jj]);
-                        }
-                    }
+                for (int j0 = 0; j0 < CH; j0 += JW) {
+                    float sx[JW];
+                    load_sx<JW>(p.s_x, ti, hcol * CH + j0, sx);
+#pragma unroll
+                    for (int jj = 0; jj < JW; ++jj)
+                        sY[(hcol * CH + j0 + jj) * 128 + r] = f32_to_bf16_bits(sx[jj] * acc[j0 + jj]);
                 }
+                named_bar_sync(4, kNumEpiWarps * 32);
+                store_staged_tile<BN>(sY, p, ti, n0, ncols, et);
             }
             u += ge - gb;
         }

@@ -365,29 +365,6 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
     *reinterpret_cast<uint4*>(out + (size_t)t * H + (size_t)c * 8) = make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-// ---------------------------------------------------------------------------
-// Split-K finish: sums the fp32 partial tiles of each output tile in CTA
-// order (fixed, so the result does not depend on timing), applies s_x and
-// rounds to bf16.  Partial slot layout: [tile][slot][col BN][row 128].
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) splitk_finish_kernel(const float* __restrict__ part,
-                                                            const float* __restrict__ s_x, int M, int N, int G,
-                                                            int bn, int n_tiles, long long Q, int slots,
-                                                            uint16_t* __restrict__ Y, int ldy) {
-    const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    if (gid >= (long long)M * N) return;
-    const int m = (int)(gid / N), n = (int)(gid % N);
-    const long long t = (long long)(m / bn) * n_tiles + n / 128;
-    const long long u0 = t * G;
-    const long long c_first = u0 / Q, c_last = (u0 + G - 1) / Q;
-    float acc = 0.0f;
-    for (long long c = c_first; c <= c_last; ++c) {
-        const long long slot = c - c_first;
-        acc += __ldg(part + (((t * slots + slot) * bn + (m % bn)) * 128 + (n % 128)));
-    }
-    Y[(size_t)m * ldy + n] = f32_to_bf16_bits(__ldg(s_x + m) * acc);
-}
-
 // Test hook: one warp waits on a barrier nobody arrives on.
 __global__ void bounded_wait_selftest_kernel(int32_t* status, unsigned long long limit_ns) {
     __shared__ __align__(8) uint64_t bar;

@@ -107,6 +107,60 @@ __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, con
     }
 }
 
+// Paired fp32 arithmetic (two independent IEEE round-to-nearest results per
+// instruction, as the scalar FADD / FFMA would give).
+__device__ __forceinline__ uint64_t f2_from_bits(uint32_t lo, uint32_t hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_splat(float a) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %1};" : "=l"(r) : "f"(a));
+    return r;
+}
+__device__ __forceinline__ void f2_split(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+// Global-memory flags between CTAs (split-K partial tiles).
+__device__ __forceinline__ void st_release_gpu_u64(unsigned long long* ptr, unsigned long long v) {
+    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(ptr), "l"(v) : "memory");
+}
+
+__device__ __forceinline__ unsigned long long ld_acquire_gpu_u64(const unsigned long long* ptr) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(ptr) : "memory");
+    return v;
+}
+
+// Waits until *ptr == v, bounded like wait_bounded; false on abort / timeout.
+__device__ __forceinline__ bool spin_until_equal_u64(const unsigned long long* ptr, unsigned long long v,
+                                                     const WaitCtx& w) {
+    if (ld_acquire_gpu_u64(ptr) == v) return true;
+    const long long t0 = clock64();
+    while (true) {
+        __nanosleep(200);
+        if (ld_acquire_gpu_u64(ptr) == v) return true;
+        if (*w.abort) return false;
+        if (clock64() - t0 > w.limit_cycles) {
+            *w.abort = 1;
+            report_status(w.status, 5);
+            return false;
+        }
+    }
+}
+
 // ----------------------------------------------------------------- TMA --
 
 // 2-D tiled tensor load into shared memory, completion counted on `bar`.
@@ -252,7 +306,10 @@ __device__ __forceinline__ void tmem_ld32<32>(uint32_t taddr, uint32_t* r) {
         : "r"(taddr));
 }
 
-// Registers -> TMEM, 32 lanes x N consecutive 32-bit columns.
+// Registers -> TMEM, 32 lanes x N consecutive 32-bit columns.  These read
+// registers only, so they carry no memory clobber (ordinary loads may be
+// scheduled across them); being volatile, they stay in order with the other
+// tcgen05 statements (fences, waits, MMAs).
 template <int N>
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r);
 
@@ -262,8 +319,7 @@ __device__ __forceinline__ void tmem_st32<16>(uint32_t taddr, const uint32_t* r)
         "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
             taddr),
         "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
-        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-        : "memory");
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]));
 }
 
 template <>
@@ -274,8 +330,7 @@ __device__ __forceinline__ void tmem_st32<32>(uint32_t taddr, const uint32_t* r)
         "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
         "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
         "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
-        "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
-        : "memory");
+        "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31]));
 }
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
@@ -287,8 +342,7 @@ __device__ __forceinline__ void tmem_fill32(uint32_t taddr, uint32_t v);
 
 template <>
 __device__ __forceinline__ void tmem_fill32<8>(uint32_t taddr, uint32_t v) {
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(taddr), "r"(v)
-                 : "memory");
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(taddr), "r"(v));
 }
 
 template <>
@@ -296,8 +350,7 @@ __device__ __forceinline__ void tmem_fill32<16>(uint32_t taddr, uint32_t v) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(
             taddr),
-        "r"(v)
-        : "memory");
+        "r"(v));
 }
 
 template <>
@@ -305,8 +358,7 @@ __device__ __forceinline__ void tmem_fill32<32>(uint32_t taddr, uint32_t v) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,"
         "%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(taddr),
-        "r"(v)
-        : "memory");
+        "r"(v));
 }
 
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {

@@ -5,6 +5,8 @@
 // launches.  Every call is asynchronous on the caller's stream and never
 // allocates; scratch lives in the caller's workspace.
 #include <atomic>
+#include <chrono>
+#include <random>
 #include <cstdint>
 #include <cstring>
 #include <cuda.h>
@@ -127,13 +129,30 @@ int pick_bn(long long rows_per_group) {
     return 128;
 }
 
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
 // Launch plan of the plain (dense) GEMM.
 struct GemmPlan {
     int bn, m_tiles, n_tiles, G, grid, slots;
     long long Q;
     bool splitk;
+    size_t flags_off;  // split-K: byte offset of the [tiles][slots] flags in the workspace
     size_t ws_bytes;
 };
+
+// Launch epochs of split-K GEMMs: nonzero 64-bit values, distinct for every
+// launch of this process, starting from a random point so that flags left
+// in a reused buffer by another process are unlikely to match.
+unsigned long long next_epoch() {
+    static std::atomic<unsigned long long> counter{[] {
+        std::random_device rd;
+        unsigned long long v = ((unsigned long long)rd() << 32) ^ rd();
+        v ^= (unsigned long long)std::chrono::steady_clock::now().time_since_epoch().count();
+        return v;
+    }()};
+    unsigned long long e = counter.fetch_add(1);
+    return e != 0 ? e : counter.fetch_add(1);
+}
 
 GemmPlan plan_gemm(int M, int N, int K, int group, int sms) {
     GemmPlan pl{};
@@ -151,7 +170,8 @@ GemmPlan plan_gemm(int M, int N, int K, int group, int sms) {
         pl.Q = (U + sms - 1) / sms;
         pl.grid = (int)((U + pl.Q - 1) / pl.Q);
         pl.slots = (int)((pl.G + pl.Q - 1) / pl.Q) + 1;
-        pl.ws_bytes = (size_t)tiles * pl.slots * pl.bn * 128 * sizeof(float);
+        pl.flags_off = align_up((size_t)tiles * pl.slots * pl.bn * 128 * sizeof(float), 256);
+        pl.ws_bytes = pl.flags_off + (size_t)tiles * pl.slots * sizeof(unsigned long long);
     } else {
         pl.Q = (long long)pl.G * waves;
         pl.grid = (int)((tiles + waves - 1) / waves);
@@ -200,8 +220,13 @@ w4a8_status gemm_impl(const int8_t* qx, const float* s_x, const uint8_t* packed,
     p.mode = pl.splitk ? kModeSplitK : kModePlain;
     p.Y = Y;
     p.ldy = ldy;
+    p.vec16 = (aligned16(Y) && ldy % 8 == 0) ? 1 : 0;
     p.partial = static_cast<float*>(workspace);
     p.slots = pl.slots;
+    if (pl.splitk) {
+        p.flags = reinterpret_cast<unsigned long long*>(static_cast<uint8_t*>(workspace) + pl.flags_off);
+        p.epoch = next_epoch();
+    }
     p.dbgP = P;
     p.n_tiles = pl.n_tiles;
     p.m_tiles = pl.m_tiles;
@@ -209,15 +234,7 @@ w4a8_status gemm_impl(const int8_t* qx, const float* s_x, const uint8_t* packed,
     p.status = dev_status;
     p.wait_ns = kDefaultWaitNs;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    st = launch_gemm(p.mode, P != nullptr, pl.bn, w->group, maps, p, pl.grid, s);
-    if (st != W4A8_OK) return st;
-    if (pl.splitk) {
-        const long long n = (long long)M * w->N;
-        splitk_finish_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(
-            static_cast<const float*>(workspace), s_x, M, w->N, pl.G, pl.bn, pl.n_tiles, pl.Q, pl.slots, Y, ldy);
-        st = last_cuda();
-    }
-    return st;
+    return launch_gemm(p.mode, P != nullptr, pl.bn, w->group, maps, p, pl.grid, s);
 }
 
 w4a8_status launch_quant(const uint16_t* X, int rows, int K, int ldx, int8_t* q, float* s_x, int32_t* rowsum,
@@ -236,7 +253,6 @@ w4a8_status launch_quant(const uint16_t* X, int rows, int K, int ldx, int8_t* q,
 
 // ------------------------------------------------------------ MoE layout --
 
-size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct MoeLayout {
     size_t mtile_off, perm, inv, qx, sx, h, qh, sh, yd, total;
@@ -472,6 +488,7 @@ w4a8_status w4a8_moe_grouped_gemm_profiled(const uint16_t* X, const float* logit
         p.mode = kModeGateUp;
         p.Y = h;
         p.ldy = I;
+        p.vec16 = 1;
         p.n_tiles = I / 64;
         p.expert_off = expert_offsets_out;
         p.mtile_off = mtile_off;
@@ -503,6 +520,7 @@ w4a8_status w4a8_moe_grouped_gemm_profiled(const uint16_t* X, const float* logit
         p.mode = kModeDown;
         p.Y = yd;
         p.ldy = H;
+        p.vec16 = 1;
         p.n_tiles = (H + 127) / 128;
         p.expert_off = expert_offsets_out;
         p.mtile_off = mtile_off;
