@@ -157,17 +157,22 @@ class LinearWorkload:
         self.Y = torch.empty(M, N, dtype=torch.bfloat16, device=self.dev)
         ws = m.w4a8_gemm_workspace_size(M, pw)
         self.ws = torch.empty(max(ws, 16), dtype=torch.uint8, device=self.dev)
+        self.lws = torch.empty(m.w4a8_linear_workspace_size(M, pw), dtype=torch.uint8, device=self.dev)
         self.splitk = ws > 0
-        self.launches_per_step = 3 if self.splitk else 2
+        self.launches_per_step = 2  # quantization + GEMM (split-K is summed inside the GEMM)
 
     def step(self, i, ev=None):
         m = self.m
+        w = self.copies[i % len(self.copies)]
+        if ev is None:
+            # the public one-call layer: the GEMM's weight streaming overlaps the quantization
+            m.w4a8_linear(self.X, w, out=self.Y, workspace=self.lws)
+            return
+        # timing replay: the same two kernels as separate calls, events around the GEMM alone
         m.w4a8_quant_act(self.X, q_out=self.q, s_out=self.s)
-        if ev is not None:
-            ev[0].record()
-        m.w4a8_gemm(self.q, self.s, self.copies[i % len(self.copies)], out=self.Y, workspace=self.ws)
-        if ev is not None:
-            ev[1].record()
+        ev[0].record()
+        m.w4a8_gemm(self.q, self.s, w, out=self.Y, workspace=self.ws)
+        ev[1].record()
 
     # metric
     def units(self):
@@ -206,8 +211,7 @@ class LinearWorkload:
 
     def e2e_step(self, i):
         self.X_dev2.copy_(self.X_pin, non_blocking=True)
-        Y = self.m.w4a8_linear(self.X_dev2, self.copies[i % len(self.copies)], out=self.Y, workspace=self.ws,
-                               q_buf=self.q, s_buf=self.s)
+        Y = self.m.w4a8_linear(self.X_dev2, self.copies[i % len(self.copies)], out=self.Y, workspace=self.lws)
         self.Y_pin.copy_(Y, non_blocking=True)
 
     # CPU oracle on a bounded sample of the same workload

@@ -179,6 +179,30 @@ W4A8_API w4a8_status w4a8_gemm(const int8_t* qx, const float* s_x,
                       void* workspace, size_t ws_bytes,
                       int32_t* dev_status, void* stream);
 
+/* Workspace bytes w4a8_linear needs for M rows. */
+W4A8_API size_t w4a8_linear_workspace_size(int M, const w4a8_wdesc* w);
+
+/*
+ * w4a8_linear — the quantized Linear layer Y = X W in one call: per-token
+ * INT8 quantization of X (as w4a8_quant_act) followed by the W4A8 GEMM (as
+ * w4a8_gemm), "Inference Quantization ch.1" §9.2 then §4.  The GEMM is
+ * launched so that its prologue and weight streaming overlap the
+ * quantization kernel (programmatic dependent launch); it reads q_x and s_x
+ * only after the quantization kernel completed.  Results are identical to
+ * w4a8_quant_act followed by w4a8_gemm.
+ * X         device bf16 [M][ldx] (rows of K = w->K used), 16-byte aligned,
+ *           ldx % 8 == 0, K <= 8192.
+ * packed, s_w, z, w: as for w4a8_gemm.
+ * Y         device bf16 [M][ldy], ldy >= N.
+ * workspace device scratch of at least w4a8_linear_workspace_size(M, w)
+ *           bytes, 16-byte aligned: holds q_x, s_x and the GEMM's split-K
+ *           partials.
+ * Errors: as w4a8_quant_act and w4a8_gemm.
+ */
+W4A8_API w4a8_status w4a8_linear(const uint16_t* X, int M, int ldx, const uint8_t* packed, const float* s_w,
+                        const uint8_t* z, const w4a8_wdesc* w, uint16_t* Y, int ldy, void* workspace,
+                        size_t ws_bytes, int32_t* dev_status, void* stream);
+
 /*
  * w4a8_gemm_debug_partials — test-only variant of w4a8_gemm that also writes
  * every exact int32 group partial P[m][g][n] (device int32 [M][G][N]) as the

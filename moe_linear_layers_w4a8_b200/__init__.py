@@ -21,7 +21,7 @@ __all__ = [
     "w4a8_pack_weights", "w4a8_pack_expert_weights", "w4a8_quant_act", "w4a8_gemm",
     "w4a8_gemm_debug_partials", "w4a8_gemm_static_scratch", "w4a8_moe_grouped_gemm", "w4a8_moe_workspace_layout",
     "w4a8_gemm_workspace_size", "w4a8_moe_workspace_size", "w4a8_get_device_status",
-    "w4a8_status_string", "w4a8_selftest_bounded_wait", "w4a8_linear", "LAYOUT_VERSION",
+    "w4a8_status_string", "w4a8_selftest_bounded_wait", "w4a8_linear", "w4a8_linear_workspace_size", "LAYOUT_VERSION",
     "STATUS",
 ]
 
@@ -110,6 +110,10 @@ def load_library():
         L.w4a8_gemm.argtypes = [P, P, P, P, P, ctypes.POINTER(WDesc), I, P, I, P, S, P, P]
         L.w4a8_gemm_static_scratch.restype = st
         L.w4a8_gemm_static_scratch.argtypes = [P, P, P, P, P, ctypes.POINTER(WDesc), I, P, I, P, P]
+        L.w4a8_linear_workspace_size.restype = S
+        L.w4a8_linear_workspace_size.argtypes = [I, ctypes.POINTER(WDesc)]
+        L.w4a8_linear.restype = st
+        L.w4a8_linear.argtypes = [P, I, I, P, P, P, ctypes.POINTER(WDesc), P, I, P, S, P, P]
         L.w4a8_gemm_debug_partials.restype = st
         L.w4a8_gemm_debug_partials.argtypes = [P, P, P, P, P, ctypes.POINTER(WDesc), I, P, I, P, P, S, P, P]
         L.w4a8_moe_grouped_gemm.restype = st
@@ -283,11 +287,28 @@ def w4a8_gemm_debug_partials(qx, s_x, w: PackedWeight, out=None, workspace=None,
     return Y, P
 
 
-def w4a8_linear(X: torch.Tensor, w: PackedWeight, out=None, workspace=None, status=None,
-                q_buf=None, s_buf=None) -> torch.Tensor:
-    """Per-token quantization of X followed by the W4A8 GEMM."""
-    q, s, _ = w4a8_quant_act(X, status=status, q_out=q_buf, s_out=s_buf)
-    return w4a8_gemm(q, s, w, out=out, workspace=workspace, status=status)
+def w4a8_linear_workspace_size(M: int, w: PackedWeight) -> int:
+    return int(load_library().w4a8_linear_workspace_size(int(M), ctypes.byref(w.desc)))
+
+
+def w4a8_linear(X: torch.Tensor, w: PackedWeight, out=None, workspace=None, status=None) -> torch.Tensor:
+    """Y bf16 [M, N] = the quantized Linear layer on X bf16 [M, K]: per-token
+    INT8 quantization then the W4A8 GEMM, in one library call."""
+    L = load_library()
+    _need_cuda(X)
+    if X.dtype != torch.bfloat16 or X.dim() != 2 or X.stride(1) != 1:
+        raise W4A8Error(1, "X must be bf16 [M, K] with unit column stride")
+    M = X.shape[0]
+    if out is None:
+        out = torch.empty(M, w.N, dtype=torch.bfloat16, device=X.device)
+    need = w4a8_linear_workspace_size(M, w)
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=X.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    code = L.w4a8_linear(_p(X), M, X.stride(0), _p(w.packed), _p(w.s_w), _p(w.z), ctypes.byref(w.desc), _p(out),
+                         out.stride(0), _p(workspace), ws_bytes, _p(status), _stream(X.device))
+    _check(code, "w4a8_linear")
+    return out
 
 
 # -------------------------------------------------------------------- MoE ---

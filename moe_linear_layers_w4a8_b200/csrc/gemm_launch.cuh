@@ -29,7 +29,17 @@ int launch_gemm_t(const GemmMaps& maps, const GemmParams& p, int grid, cudaStrea
             return 6;
         attr_done.fetch_or(bit);
     }
-    kern<<<grid, kGemmThreads, C::SMEM, stream>>>(maps.act, maps.sw, maps.z, p);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kGemmThreads);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = p.pdl ? 1 : 0;
+    if (cudaLaunchKernelEx(&cfg, kern, maps.act, maps.sw, maps.z, p) != cudaSuccess) return 6;
     return cudaGetLastError() == cudaSuccess ? 0 : 6;
 }
 

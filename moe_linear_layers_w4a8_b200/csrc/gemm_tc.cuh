@@ -90,6 +90,7 @@ struct GemmParams {
     int32_t* status;
     unsigned long long wait_ns;
     int vec16;                   // Y and ldy allow 16-byte row stores
+    int pdl;                     // launched with programmatic stream serialization
 };
 
 constexpr int kGemmThreads = 512;  // 4 unpack, 8 epilogue, 2 producer, 1 MMA, 1 spare warp
@@ -349,6 +350,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     const WaitCtx wc{abort_flag, p.status, wait_cycles_for_ns(p.wait_ns)};
+    // Launched right behind the kernel that produces the activations
+    // (programmatic dependent launch): only the packed weights, scales and
+    // zero-points may be read before griddepcontrol.wait.  The grouped MoE
+    // modes need the dispatch offsets to plan their ranges, so all threads
+    // wait; the dense modes wait in the activation producer and epilogue.
+    if constexpr (MODE == kModeGateUp || MODE == kModeDown) pdl_wait_prerequisites();
 
     long long u0, u1, Q;
     cta_units<MODE>(p, u0, u1, Q);
@@ -402,6 +409,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     } else if (warp == kWarpAct) {
         // ------------------------- producer: activation tiles, group scales --
         if (lane == 0) {
+            if constexpr (MODE == kModePlain || MODE == kModeSplitK) pdl_wait_prerequisites();
             Ring ra, rw;
             long long na = 0, nw = 0;
             bool ok = true;
@@ -600,6 +608,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         __syncwarp();
         if (lane == 0)
             for (int b = 0; b < NS; ++b) mbar_arrive(&ready[b]);
+        // s_x, Y and the split-K workspace are touched only after this
+        if constexpr (MODE == kModePlain || MODE == kModeSplitK) pdl_wait_prerequisites();
 
         bool ok = true;
         Ring rw, rs;

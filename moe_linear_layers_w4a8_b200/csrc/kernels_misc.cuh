@@ -29,6 +29,10 @@ __global__ void __launch_bounds__(kQuantThreads) quant_act_kernel(
     const uint16_t* __restrict__ X, int K, int ldx, int8_t* __restrict__ q, float* __restrict__ s_x,
     int32_t* __restrict__ rowsum, int group, const int32_t* __restrict__ dest, int dest_k,
     int32_t* status) {
+    // A GEMM launched after this kernel with programmatic stream serialization
+    // may start its prologue and weight streaming now; it waits for this
+    // grid's completion before it reads q / s_x.
+    pdl_launch_dependents();
     const int m = blockIdx.x;
     const int tid = threadIdx.x;
     const int nchunk = K >> 3;

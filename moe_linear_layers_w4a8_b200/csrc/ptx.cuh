@@ -133,6 +133,16 @@ __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
     return d;
 }
 
+// Programmatic dependent launch.  launch_dependents: the next kernel of the
+// stream (launched with programmatic stream serialization) may start now.
+// wait_prerequisites: block until the preceding kernel has completed and its
+// memory operations are visible; a kernel launched without the attribute
+// returns at once.
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait_prerequisites() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Global-memory flags between CTAs (split-K partial tiles).
 __device__ __forceinline__ void st_release_gpu_u64(unsigned long long* ptr, unsigned long long v) {
     asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(ptr), "l"(v) : "memory");

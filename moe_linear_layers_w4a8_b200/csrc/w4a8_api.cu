@@ -192,7 +192,7 @@ w4a8_status check_wdesc(const w4a8_wdesc* w) {
 
 w4a8_status gemm_impl(const int8_t* qx, const float* s_x, const uint8_t* packed, const float* s_w,
                       const uint8_t* z, const w4a8_wdesc* w, int M, uint16_t* Y, int ldy, int32_t* P,
-                      void* workspace, size_t ws_bytes, int32_t* dev_status, void* stream) {
+                      void* workspace, size_t ws_bytes, int32_t* dev_status, void* stream, bool pdl = false) {
     w4a8_status st = check_wdesc(w);
     if (st != W4A8_OK) return st;
     if (M < 0 || !Y || ldy < w->N) return W4A8_ERR_INVALID_ARG;
@@ -221,6 +221,7 @@ w4a8_status gemm_impl(const int8_t* qx, const float* s_x, const uint8_t* packed,
     p.Y = Y;
     p.ldy = ldy;
     p.vec16 = (aligned16(Y) && ldy % 8 == 0) ? 1 : 0;
+    p.pdl = pdl ? 1 : 0;
     p.partial = static_cast<float*>(workspace);
     p.slots = pl.slots;
     if (pl.splitk) {
@@ -295,6 +296,20 @@ w4a8_status check_moe(int T, int E, int topk, const w4a8_wdesc* w1, const w4a8_w
 
 // ===================================================================== ABI ==
 
+// Workspace of w4a8_linear: q_x [M][K] int8, s_x [M] fp32, then the GEMM's own.
+struct LinearLayout {
+    size_t qx, sx, gemm, total;
+};
+
+LinearLayout linear_layout(int M, const w4a8_wdesc* w) {
+    LinearLayout L{};
+    L.qx = 0;
+    L.sx = align_up((size_t)M * w->K, 256);
+    L.gemm = align_up(L.sx + sizeof(float) * (size_t)M, 256);
+    L.total = L.gemm + plan_gemm(M, w->N, w->K, w->group, sm_count_current()).ws_bytes;
+    return L;
+}
+
 extern "C" {
 
 int w4a8_abi_version(void) { return W4A8_ABI_VERSION; }
@@ -321,6 +336,11 @@ size_t w4a8_packed_bytes(int K, int N) {
 size_t w4a8_gemm_workspace_size(int M, const w4a8_wdesc* w) {
     if (M <= 0 || check_wdesc(w) != W4A8_OK) return 0;
     return plan_gemm(M, w->N, w->K, w->group, sm_count_current()).ws_bytes;
+}
+
+size_t w4a8_linear_workspace_size(int M, const w4a8_wdesc* w) {
+    if (M <= 0 || check_wdesc(w) != W4A8_OK) return 0;
+    return linear_layout(M, w).total;
 }
 
 size_t w4a8_moe_workspace_size(int T, int E, int topk, const w4a8_wdesc* w1, const w4a8_wdesc* w2) {
@@ -394,6 +414,30 @@ w4a8_status w4a8_gemm(const int8_t* qx, const float* s_x, const uint8_t* packed,
                       const w4a8_wdesc* w, int M, uint16_t* Y, int ldy, void* workspace, size_t ws_bytes,
                       int32_t* dev_status, void* stream) {
     return gemm_impl(qx, s_x, packed, s_w, z, w, M, Y, ldy, nullptr, workspace, ws_bytes, dev_status, stream);
+}
+
+w4a8_status w4a8_linear(const uint16_t* X, int M, int ldx, const uint8_t* packed, const float* s_w,
+                        const uint8_t* z, const w4a8_wdesc* w, uint16_t* Y, int ldy, void* workspace,
+                        size_t ws_bytes, int32_t* dev_status, void* stream) {
+    w4a8_status st = check_wdesc(w);
+    if (st != W4A8_OK) return st;
+    if (M < 0 || !Y || ldy < w->N) return W4A8_ERR_INVALID_ARG;
+    if (M == 0) return W4A8_OK;
+    if (!X || ldx < w->K) return W4A8_ERR_INVALID_ARG;
+    if (w->K % 8 != 0 || ldx % 8 != 0 || !aligned16(X) || w->K > 8192) return W4A8_ERR_UNSUPPORTED_SHAPE;
+    const LinearLayout L = linear_layout(M, w);
+    if (!workspace || ws_bytes < L.total || !aligned16(workspace)) return W4A8_ERR_WORKSPACE;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    int8_t* qx = reinterpret_cast<int8_t*>(ws + L.qx);
+    float* sx = reinterpret_cast<float*>(ws + L.sx);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    st = launch_quant(X, M, w->K, ldx, qx, sx, nullptr, 0, nullptr, 0, dev_status, s);
+    if (st != W4A8_OK) return st;
+    // The GEMM follows our quantization kernel, which triggers its dependents
+    // at entry: launched with programmatic stream serialization, its prologue
+    // and weight streaming overlap the quantization.
+    return gemm_impl(qx, sx, packed, s_w, z, w, M, Y, ldy, nullptr, ws + L.gemm, ws_bytes - L.gemm, dev_status,
+                     stream, true);
 }
 
 w4a8_status w4a8_gemm_debug_partials(const int8_t* qx, const float* s_x, const uint8_t* packed, const float* s_w,

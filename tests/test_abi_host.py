@@ -109,6 +109,20 @@ def test_gemm_rejects_bad_args(lib):
                                         None, 0, None, None) == 1
 
 
+def test_linear_sizes_and_rejections(lib):
+    d = _desc()
+    need = lib.w4a8_linear_workspace_size(16, ctypes.byref(d))
+    assert need >= 16 * 512 + 16 * 4                       # q_x and s_x at least
+    assert lib.w4a8_linear_workspace_size(0, ctypes.byref(d)) == 0
+    bad = _desc(layout_version=2)
+    assert lib.w4a8_linear(FAKE, 16, 512, FAKE, FAKE, None, ctypes.byref(bad), FAKE, 512, FAKE, need, None, None) == 3
+    assert lib.w4a8_linear(FAKE, 16, 512, FAKE, FAKE, None, ctypes.byref(d), FAKE, 512, FAKE, need - 1, None, None) == 7
+    assert lib.w4a8_linear(FAKE, 16, 100, FAKE, FAKE, None, ctypes.byref(d), FAKE, 512, FAKE, need, None, None) == 1
+    assert lib.w4a8_linear(FAKE, 16, 512, FAKE, FAKE, None, ctypes.byref(d), FAKE, 100, FAKE, need, None, None) == 1
+    assert lib.w4a8_linear(FAKE, -1, 512, FAKE, FAKE, None, ctypes.byref(d), FAKE, 512, FAKE, need, None, None) == 1
+    assert lib.w4a8_linear(FAKE, 0, 512, FAKE, FAKE, None, ctypes.byref(d), FAKE, 512, FAKE, 0, None, None) == 0
+
+
 def test_pack_rejects_bad_args(lib):
     d = _desc()
     # K not a multiple of the group ("groups cannot cross rows")

@@ -200,3 +200,23 @@ def test_bounded_wait_reports_timeout(m):
     # the context is still usable afterwards
     x = torch.ones(4, device="cuda")
     assert float(x.sum()) == 4.0
+
+
+@pytest.mark.parametrize("M,K,N,group,sym", [(32, 4096, 14336, 128, True), (1, 4096, 14336, 128, True),
+                                             (300, 2048, 1024, 128, True), (17, 1024, 512, 64, False)])
+def test_linear_one_call_equals_quant_then_gemm(m, M, K, N, group, sym):
+    """w4a8_linear (quantization and GEMM in one call, the GEMM launched to
+    overlap the quantization) gives bit for bit what the two calls give."""
+    inp = gen_linear(M, K, N, seed=M + N)
+    W = inp.W if sym else _weights(K, N, 5, False)
+    pw = m.w4a8_pack_weights(W.cuda(), group, sym)
+    X = inp.X.cuda()
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    Y1 = m.w4a8_linear(X, pw, status=st)
+    Y1b = m.w4a8_linear(X, pw, status=st)  # again: the split-K flags of the first call must not leak
+    q, s, _ = m.w4a8_quant_act(X)
+    Y2 = m.w4a8_gemm(q, s, pw)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert np.array_equal(bits(Y1), bits(Y2))
+    assert np.array_equal(bits(Y1b), bits(Y2))
