@@ -316,39 +316,47 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    if (threadIdx.x == 0) {
-        for (int i = 0; i < C::SPC; ++i) {
-            mbar_init(&p_full[i], 1);
-            mbar_init(&p_empty[i], kUnpackWarps);
+    // Start-up: the packed-code producer initialises every barrier and starts
+    // streaming weights at once; it only arrives on the start barrier, while
+    // the other warps wait there (for the barriers and the TMEM allocation).
+    if (warp == kWarpPack) {
+        if (lane == 0) {
+            for (int i = 0; i < C::SPC; ++i) {
+                mbar_init(&p_full[i], 1);
+                mbar_init(&p_empty[i], kUnpackWarps);
+            }
+            for (int i = 0; i < C::SAC; ++i) {
+                mbar_init(&act_full[i], 1);
+                mbar_init(&act_empty[i], 1);
+            }
+            for (int i = 0; i < C::SWC; ++i) {
+                mbar_init(&sw_full[i], 1);
+                mbar_init(&sw_empty[i], kNumEpiWarps);
+            }
+            for (int i = 0; i < NS; ++i) {
+                mbar_init(&ready[i], kUnpackWarps + kNumEpiWarps);
+                mbar_init(&done[i], 1);
+            }
+            mbar_init(drain, 1);
+            *abort_flag = 0;
+            fence_mbar_init();
+            fence_proxy_async_smem();
+            prefetch_tmap(&tmap_act);
+            prefetch_tmap(&tmap_sw);
+            if (!p.symmetric) prefetch_tmap(&tmap_z);
         }
-        for (int i = 0; i < C::SAC; ++i) {
-            mbar_init(&act_full[i], 1);
-            mbar_init(&act_empty[i], 1);
+        __syncwarp();
+        named_bar_arrive(5, kGemmThreads);
+    } else {
+        if (warp == kWarpMma) {
+            tmem_alloc(tmem_slot, C::TMEM_COLS);
+            tmem_relinquish();
         }
-        for (int i = 0; i < C::SWC; ++i) {
-            mbar_init(&sw_full[i], 1);
-            mbar_init(&sw_empty[i], kNumEpiWarps);
-        }
-        for (int i = 0; i < NS; ++i) {
-            mbar_init(&ready[i], kUnpackWarps + kNumEpiWarps);
-            mbar_init(&done[i], 1);
-        }
-        mbar_init(drain, 1);
-        *abort_flag = 0;
-        fence_mbar_init();
-        fence_proxy_async_smem();
-        prefetch_tmap(&tmap_act);
-        prefetch_tmap(&tmap_sw);
-        if (!p.symmetric) prefetch_tmap(&tmap_z);
+        tc_fence_before();
+        named_bar_sync(5, kGemmThreads);
+        tc_fence_after();
     }
-    if (warp == kWarpMma) {
-        tmem_alloc(tmem_slot, C::TMEM_COLS);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem_base = *tmem_slot;
+    const uint32_t tmem_base = (warp == kWarpPack) ? 0u : *tmem_slot;  // the producer never touches TMEM
     const WaitCtx wc{abort_flag, p.status, wait_cycles_for_ns(p.wait_ns)};
     // Launched right behind the kernel that produces the activations
     // (programmatic dependent launch): only the packed weights, scales and

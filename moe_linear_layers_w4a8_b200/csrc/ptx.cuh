@@ -375,6 +375,11 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// Counts the calling threads on named barrier `id` without waiting.
+__device__ __forceinline__ void named_bar_arrive(int id, int nthreads) {
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 // Named barrier that also ORs a predicate over all participating threads;
 // every thread gets the same result.
 __device__ __forceinline__ bool named_bar_or(int id, int nthreads, bool pred) {
