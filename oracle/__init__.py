@@ -299,7 +299,7 @@ def moe_forward(X_bf16, logits, topk, experts_w1, experts_w2, group):
     tok = perm // topk
     q_perm = qx[tok]
     s_perm = sx[tok]
-    I2 = experts_w1[0][0].shape[0]
+    I2 = next(w[0] for w in experts_w1 if w[0] is not None).shape[0]  # any expert present
     I = I2 // 2
     H_gu = np.zeros((T * topk, I2), dtype=np.float64)
     P1 = [None] * E
