@@ -114,6 +114,10 @@ GEMM_CASES = [
     (64, 256, 64, 128, True),       # a single half tile
     (513, 512, 1024, 128, True),    # many tiles, ragged last row block
     (33, 4096, 1024, 128, True),    # BN=64, split-K
+    (20, 128, 256, 128, True),      # one group (G = 1)
+    (9, 64, 192, 64, False),        # one group, asymmetric, half tile
+    (8, 4096, 1024, 128, True),     # split-K: 8 tiles over the SMs, every tile summed from ~16 CTAs
+    (5, 2048, 1024, 64, False),     # split-K, asymmetric g=64, ragged M
 ]
 
 
@@ -220,3 +224,47 @@ def test_linear_one_call_equals_quant_then_gemm(m, M, K, N, group, sym):
     assert int(st.item()) == 0
     assert np.array_equal(bits(Y1), bits(Y2))
     assert np.array_equal(bits(Y1b), bits(Y2))
+
+
+def test_gemm_zero_rows_and_zero_groups(m):
+    """All-zero activation rows give s_x = 0 and exactly zero outputs; an
+    all-zero weight group gives s_w = 0 and contributes nothing (the zero-scale
+    reading of "Quantization: formats, error and the real execution path")."""
+    M, K, N, g = 24, 1024, 384, 128
+    inp = gen_linear(M, K, N, seed=77)
+    X = inp.X.clone()
+    X[[0, 5, 23]] = 0
+    W = inp.W.clone()
+    W[128:256, 64:80] = 0          # group 1 of columns 64..79
+    W[:, 300] = 0                   # every group of column 300
+    pw = m.w4a8_pack_weights(W.cuda(), g, True)
+    codes, s, z, _ = O.quant_weights(W.numpy(), g, True)
+    assert (s[1, 64:80] == 0).all() and (s[:, 300] == 0).all()
+    st = m.new_status("cuda")
+    q, sx, _ = m.w4a8_quant_act(X.cuda(), status=st)
+    Y, P = m.w4a8_gemm_debug_partials(q, sx, pw, status=st)
+    assert m.w4a8_get_device_status(st) == 0
+    qo, so, _, _ = O.quant_act(bits(X))
+    assert np.array_equal(P.cpu().numpy(), O.partials(qo, codes, None, g))
+    Ye, A = O.scale_partials(O.partials(qo, codes, None, g), so, s)
+    check_bf16(bits(Y), Ye, A)
+    Yb = bits(Y)
+    assert (Yb[[0, 5, 23]] & 0x7FFF == 0).all()
+    assert (Yb[:, 300] & 0x7FFF == 0).all()
+
+
+@pytest.mark.parametrize("M", [3, 33, 130])
+def test_gemm_strided_output(m, M):
+    """Y with a row pitch of N + 3 elements (no 16-byte row stores) holds the
+    same bits as a contiguous Y, and the padding is left untouched."""
+    K, N = 1024, 512
+    inp = gen_linear(M, K, N, seed=M)
+    pw = m.w4a8_pack_weights(inp.W.cuda(), 128, True)
+    q, sx, _ = m.w4a8_quant_act(inp.X.cuda())
+    Yc = m.w4a8_gemm(q, sx, pw)
+    big = torch.full((M, N + 3), -7.0, dtype=torch.bfloat16, device="cuda")
+    Ys = m.w4a8_gemm(q, sx, pw, out=big[:, :N])
+    torch.cuda.synchronize()
+    assert Ys.stride(0) == N + 3
+    assert np.array_equal(bits(Ys), bits(Yc))
+    assert (big[:, N:] == -7.0).all()

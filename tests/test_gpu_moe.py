@@ -171,6 +171,7 @@ SMALL = [
     (33, 128, 4, 4, 64, 64, True, 1.1),     # topk == E: every token visits every expert
     (200, 256, 64, 6, 128, 128, True, 1.1),  # many experts with 0 tokens
     (1, 256, 8, 2, 128, 64, False, None),    # a single token
+    (40, 128, 512, 16, 64, 64, True, 1.1),   # the largest E and top-k the dispatch supports
 ]
 
 
