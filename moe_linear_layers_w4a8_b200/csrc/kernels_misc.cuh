@@ -126,6 +126,96 @@ __global__ void __launch_bounds__(kQuantThreads) quant_act_kernel(
     }
 }
 
+// The same quantization with one warp per row (8 rows per CTA): no block-wide
+// reduction, and many more rows in flight per SM, for launches with many rows
+// of at most 4096 elements.  Lane l holds chunks l, l + 32, ... of its row, so
+// the per-group code sums are segmented shuffles over 8 or 16 lanes exactly
+// as above; every value is computed by the same operations.
+constexpr int kQuantRowsPerCta = 8;
+
+template <int CPL>
+__global__ void __launch_bounds__(32 * kQuantRowsPerCta) quant_act_rows_kernel(
+    const uint16_t* __restrict__ X, int rows, int K, int ldx, int8_t* __restrict__ q, float* __restrict__ s_x,
+    int32_t* __restrict__ rowsum, int group, const int32_t* __restrict__ dest, int dest_k, int32_t* status) {
+    pdl_launch_dependents();
+    const int lane = threadIdx.x & 31;
+    const int m = blockIdx.x * kQuantRowsPerCta + (threadIdx.x >> 5);
+    if (m >= rows) return;  // warp-uniform
+    const int nchunk = K >> 3;
+    const uint4* xr = reinterpret_cast<const uint4*>(X + (size_t)m * ldx);
+
+    uint4 raw[CPL];
+    float amax = 0.0f;
+    uint32_t bad = 0;
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) {
+        const int c = i * 32 + lane;
+        raw[i] = make_uint4(0, 0, 0, 0);
+        if (c < nchunk) raw[i] = __ldg(xr + c);
+    }
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) {
+        const uint32_t w[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+            const uint32_t lo = w[h] & 0xFFFFu, hi = w[h] >> 16;
+            bad |= ((lo & 0x7F80u) == 0x7F80u) | ((hi & 0x7F80u) == 0x7F80u);
+            amax = fmaxf(amax, fabsf(bf16_bits_to_f32(lo)));
+            amax = fmaxf(amax, fabsf(bf16_bits_to_f32(hi)));
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
+        bad |= __shfl_xor_sync(0xFFFFFFFFu, bad, off);
+    }
+    const float s = __fdiv_rn(amax, 127.0f);
+    const float d = (s > 0.0f) ? s : 1.0f;
+
+    const int nrows_out = dest ? dest_k : 1;
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) {
+        const int c = i * 32 + lane;
+        const bool live = c < nchunk;
+        const uint32_t w[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
+        uint32_t packed[2] = {0u, 0u};
+        int32_t csum = 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const uint32_t bits = (e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xFFFFu);
+            float t = rintf(__fdiv_rn(bf16_bits_to_f32(bits), d));
+            t = fminf(fmaxf(t, -127.0f), 127.0f);
+            const int qi = (int)t;
+            csum += qi;
+            packed[e >> 2] |= ((uint32_t)(qi & 0xFF)) << (8 * (e & 3));
+        }
+        if (live) {
+            for (int j = 0; j < nrows_out; ++j) {
+                const int row = dest ? dest[(size_t)m * dest_k + j] : m;
+                *reinterpret_cast<uint2*>(q + (size_t)row * K + (size_t)c * 8) = make_uint2(packed[0], packed[1]);
+            }
+        }
+        if (rowsum) {
+            const int lanes = group >> 3;
+            for (int off = lanes >> 1; off > 0; off >>= 1) csum += __shfl_xor_sync(0xFFFFFFFFu, csum, off);
+            if (live && (c % lanes) == 0) {
+                const int G = K / group;
+                for (int j = 0; j < nrows_out; ++j) {
+                    const int row = dest ? dest[(size_t)m * dest_k + j] : m;
+                    rowsum[(size_t)row * G + c / lanes] = csum;
+                }
+            }
+        }
+    }
+    if (lane == 0) {
+        for (int j = 0; j < nrows_out; ++j) {
+            const int row = dest ? dest[(size_t)m * dest_k + j] : m;
+            s_x[row] = s;
+        }
+        if (bad) report_status(status, kStatusNonfinite);
+    }
+}
+
 // ---------------------------------------------------------------------------
 // Offline group-wise 4-bit quantization and packing ("Quantization: formats,
 // error and the real execution path", sections "Basic mapping" and

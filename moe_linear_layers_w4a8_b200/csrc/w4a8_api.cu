@@ -241,6 +241,20 @@ w4a8_status gemm_impl(const int8_t* qx, const float* s_x, const uint8_t* packed,
 w4a8_status launch_quant(const uint16_t* X, int rows, int K, int ldx, int8_t* q, float* s_x, int32_t* rowsum,
                          int group, const int32_t* dest, int dest_k, int32_t* status, cudaStream_t s) {
     if (rows == 0) return W4A8_OK;
+    if (rows >= 8192 && K <= 2048) {
+        // very many short rows (measured: faster there, slower for fewer or
+        // longer rows): one warp per row, chunks per lane rounded up to a built size
+        const int need = (K / 8 + 31) / 32;
+        const int cpl = need <= 1 ? 1 : need <= 2 ? 2 : need <= 4 ? 4 : need <= 6 ? 6 : need <= 8 ? 8 : need <= 12 ? 12 : 16;
+        const unsigned blocks = (unsigned)((rows + kQuantRowsPerCta - 1) / kQuantRowsPerCta);
+        const unsigned threads = 32 * kQuantRowsPerCta;
+        switch (cpl) {
+#define W4A8_QROWS(n) case n: quant_act_rows_kernel<n><<<blocks, threads, 0, s>>>(X, rows, K, ldx, q, s_x, rowsum, group, dest, dest_k, status); break;
+            W4A8_QROWS(1) W4A8_QROWS(2) W4A8_QROWS(4) W4A8_QROWS(6) W4A8_QROWS(8) W4A8_QROWS(12) W4A8_QROWS(16)
+#undef W4A8_QROWS
+        }
+        return last_cuda();
+    }
     const int cpt = (K / 8 + kQuantThreads - 1) / kQuantThreads;
     switch (cpt) {
         case 1: quant_act_kernel<1><<<rows, kQuantThreads, 0, s>>>(X, K, ldx, q, s_x, rowsum, group, dest, dest_k, status); break;

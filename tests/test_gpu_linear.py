@@ -35,7 +35,9 @@ def _weights(K, N, seed, symmetric, outlier_p=0.0):
 
 # ----------------------------------------------------------------- quant ---
 
-@pytest.mark.parametrize("M,K", [(16, 512), (1, 4096), (37, 1408), (8, 7168), (300, 2048), (3, 8), (2, 8192)])
+@pytest.mark.parametrize("M,K", [(16, 512), (1, 4096), (37, 1408), (8, 7168), (300, 2048), (3, 8), (2, 8192),
+                                 (1000, 1408), (129, 2056), (70, 4104),
+                                 (8192, 8), (8200, 512), (8193, 1408), (9000, 2048)])  # one warp per row
 def test_quant_act_bit_exact(m, M, K):
     inp = gen_linear(M, K, 64, seed=M + K, n_outliers=min(8, K // 2), outlier_scale=50.0)
     st = m.new_status("cuda")
@@ -67,9 +69,10 @@ def test_quant_act_strided_rows_zero_rows_and_ties(m):
 
 
 @pytest.mark.parametrize("bad", [0x7FC0, 0x7F80, 0xFF80])
-def test_quant_act_flags_nonfinite(m, bad):
-    X = torch.ones(3, 256, dtype=torch.bfloat16)
-    X.view(torch.int16)[1, 17] = np.int16(np.uint16(bad).view(np.int16))
+@pytest.mark.parametrize("rows", [3, 8200])  # one CTA per row / one warp per row
+def test_quant_act_flags_nonfinite(m, bad, rows):
+    X = torch.ones(rows, 256, dtype=torch.bfloat16)
+    X.view(torch.int16)[rows - 2, 17] = np.int16(np.uint16(bad).view(np.int16))
     st = m.new_status("cuda")
     m.w4a8_quant_act(X.cuda(), status=st)
     assert m.w4a8_get_device_status(st) == 4
