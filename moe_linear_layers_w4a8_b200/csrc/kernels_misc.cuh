@@ -425,6 +425,111 @@ __global__ void __launch_bounds__(kDispatchThreads) dispatch_kernel(const int32_
     }
 }
 
+// The same dispatch spread over many CTAs, for many tokens: each CTA owns a
+// contiguous run of `tpc` tokens.  (1) every CTA counts its pairs per
+// expert; (2) one CTA turns the counts into the expert offsets, the m-tile
+// prefix and every CTA's first position per expert (written over the
+// counts); (3) every CTA places its pairs exactly as dispatch_kernel does,
+// chunk by chunk from its own first positions.  Positions stay ordered by
+// (expert, token, slot), so the output equals dispatch_kernel's.
+__global__ void __launch_bounds__(kDispatchThreads) dispatch_count_kernel(const int32_t* __restrict__ idx, int T,
+                                                                          int E, int topk, int tpc,
+                                                                          int32_t* __restrict__ cnt_g) {
+    __shared__ int32_t cnt[kMaxExperts];
+    const int c = blockIdx.x, tid = threadIdx.x;
+    for (int e = tid; e < E; e += kDispatchThreads) cnt[e] = 0;
+    __syncthreads();
+    const long long p0 = (long long)c * tpc * topk;
+    const long long p1 = (long long)min((long long)(c + 1) * tpc, (long long)T) * topk;
+    for (long long i = p0 + tid; i < p1; i += kDispatchThreads) atomicAdd(&cnt[idx[i]], 1);
+    __syncthreads();
+    for (int e = tid; e < E; e += kDispatchThreads) cnt_g[(size_t)c * E + e] = cnt[e];
+}
+
+constexpr int kDispatchScanThreads = kMaxExperts;  // one thread per expert
+
+__global__ void __launch_bounds__(kDispatchScanThreads) dispatch_scan_kernel(int32_t* __restrict__ cnt_g, int C,
+                                                                            int E, int bn,
+                                                                            int32_t* __restrict__ offsets,
+                                                                            int32_t* __restrict__ mtile_off) {
+    __shared__ int32_t tot[kMaxExperts], til[kMaxExperts];
+    const int e = threadIdx.x;
+    int32_t total = 0;
+    if (e < E)
+        for (int c = 0; c < C; ++c) total += cnt_g[(size_t)c * E + e];
+    const int32_t tiles = (total + bn - 1) / bn;
+    tot[e] = total;  // zero for e >= E
+    til[e] = tiles;
+    __syncthreads();
+    for (int off = 1; off < kMaxExperts; off <<= 1) {  // inclusive scans over the experts
+        const int32_t a = (e >= off) ? tot[e - off] : 0;
+        const int32_t b = (e >= off) ? til[e - off] : 0;
+        __syncthreads();
+        tot[e] += a;
+        til[e] += b;
+        __syncthreads();
+    }
+    if (e < E) {
+        const int32_t first = tot[e] - total;
+        offsets[e] = first;
+        mtile_off[e] = til[e] - tiles;
+        int32_t run = first;
+        for (int c = 0; c < C; ++c) {
+            const int32_t v = cnt_g[(size_t)c * E + e];
+            cnt_g[(size_t)c * E + e] = run;  // the CTA's first position for this expert
+            run += v;
+        }
+        if (e == E - 1) {
+            offsets[E] = tot[e];
+            mtile_off[E] = til[e];
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kDispatchThreads) dispatch_scatter_kernel(const int32_t* __restrict__ idx, int T,
+                                                                            int E, int topk, int tpc,
+                                                                            const int32_t* __restrict__ base_g,
+                                                                            int32_t* __restrict__ perm,
+                                                                            int32_t* __restrict__ inv) {
+    __shared__ int32_t cnt[kMaxExperts];
+    __shared__ int32_t base[kMaxExperts];
+    __shared__ uint32_t bits[kDispatchThreads / 32][kMaxExperts];
+    __shared__ int32_t wpre[kDispatchThreads / 32][kMaxExperts];
+    const int c = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    for (int e = tid; e < E; e += kDispatchThreads) base[e] = base_g[(size_t)c * E + e];
+    __syncthreads();
+    const int t_end = (int)min((long long)(c + 1) * tpc, (long long)T);
+    for (int t0 = c * tpc; t0 < t_end; t0 += kDispatchThreads) {
+        for (int e = lane; e < E; e += 32) bits[warp][e] = 0u;
+        __syncthreads();
+        const int t = t0 + tid;
+        if (t < t_end)
+            for (int j = 0; j < topk; ++j) atomicOr(&bits[warp][idx[(size_t)t * topk + j]], 1u << lane);
+        __syncthreads();
+        for (int e = tid; e < E; e += kDispatchThreads) {
+            int32_t run = 0;
+            for (int w = 0; w < kDispatchThreads / 32; ++w) {
+                wpre[w][e] = run;
+                run += __popc(bits[w][e]);
+            }
+            cnt[e] = run;
+        }
+        __syncthreads();
+        if (t < t_end) {
+            const uint32_t lt = (1u << lane) - 1u;
+            for (int j = 0; j < topk; ++j) {
+                const int e = idx[(size_t)t * topk + j];
+                const int32_t pos = base[e] + wpre[warp][e] + __popc(bits[warp][e] & lt);
+                inv[(size_t)t * topk + j] = pos;
+                perm[pos] = t * topk + j;
+            }
+        }
+        __syncthreads();
+        for (int e = tid; e < E; e += kDispatchThreads) base[e] += cnt[e];
+        __syncthreads();
+    }
+}
+
 // ---------------------------------------------------------------------------
 // Weighted combine ("Kimi 2.7 MoE, 4-bit storage to INT8" §4.3-4.4 step 5):
 // out[t] = sum_j p[t,j] * y[inv(t,j)], fp32 in slot order, one bf16 rounding.

@@ -241,9 +241,10 @@ w4a8_status gemm_impl(const int8_t* qx, const float* s_x, const uint8_t* packed,
 w4a8_status launch_quant(const uint16_t* X, int rows, int K, int ldx, int8_t* q, float* s_x, int32_t* rowsum,
                          int group, const int32_t* dest, int dest_k, int32_t* status, cudaStream_t s) {
     if (rows == 0) return W4A8_OK;
-    if (rows >= 8192 && K <= 2048) {
-        // very many short rows (measured: faster there, slower for fewer or
-        // longer rows): one warp per row, chunks per lane rounded up to a built size
+    if (rows >= 8192 && K <= 1536) {
+        // very many short rows (measured on B200: 24576 x 1408 80 -> 57 us;
+        // slower for fewer or longer rows, e.g. 65536 x 2048): one warp per
+        // row, chunks per lane rounded up to a built size
         const int need = (K / 8 + 31) / 32;
         const int cpl = need <= 1 ? 1 : need <= 2 ? 2 : need <= 4 ? 4 : need <= 6 ? 6 : need <= 8 ? 8 : need <= 12 ? 12 : 16;
         const unsigned blocks = (unsigned)((rows + kQuantRowsPerCta - 1) / kQuantRowsPerCta);
@@ -270,8 +271,18 @@ w4a8_status launch_quant(const uint16_t* X, int rows, int K, int ldx, int8_t* q,
 
 
 struct MoeLayout {
-    size_t mtile_off, perm, inv, qx, sx, h, qh, sh, yd, total;
+    size_t mtile_off, perm, inv, qx, sx, h, qh, sh, yd, dcnt, total;
 };
+
+// Dispatch over several CTAs: tokens per CTA (a multiple of 256, at most 1024 CTAs).
+int dispatch_tokens_per_cta(int T) {
+    const int chunks = (T + kDispatchThreads - 1) / kDispatchThreads;
+    return kDispatchThreads * ((chunks + 1023) / 1024);
+}
+int dispatch_ctas(int T) {
+    const int tpc = dispatch_tokens_per_cta(T);
+    return (T + tpc - 1) / tpc;
+}
 
 MoeLayout moe_layout(int T, int E, int topk, int H, int I) {
     MoeLayout L{};
@@ -286,6 +297,7 @@ MoeLayout moe_layout(int T, int E, int topk, int H, int I) {
     L.qh = o;        o = align_up(o + R * I, 256);
     L.sh = o;        o = align_up(o + sizeof(float) * R, 256);
     L.yd = o;        o = align_up(o + 2 * R * H, 256);
+    L.dcnt = o;      o = align_up(o + sizeof(int32_t) * (size_t)dispatch_ctas(T) * E, 256);
     L.total = o;
     return L;
 }
@@ -521,8 +533,18 @@ w4a8_status w4a8_moe_grouped_gemm_profiled(const uint16_t* X, const float* logit
     }
     // 2. dispatch
     if (!mark(1)) return W4A8_ERR_CUDA;
-    dispatch_kernel<<<1, kDispatchThreads, 0, s>>>(topk_idx_out, T, E, topk, bn, expert_offsets_out, mtile_off,
-                                                   perm, inv);
+    if (T <= kDispatchThreads) {
+        dispatch_kernel<<<1, kDispatchThreads, 0, s>>>(topk_idx_out, T, E, topk, bn, expert_offsets_out, mtile_off,
+                                                       perm, inv);
+    } else {
+        const int tpc = dispatch_tokens_per_cta(T), C = dispatch_ctas(T);
+        int32_t* dcnt = reinterpret_cast<int32_t*>(ws + L.dcnt);
+        dispatch_count_kernel<<<C, kDispatchThreads, 0, s>>>(topk_idx_out, T, E, topk, tpc, dcnt);
+        if ((st = last_cuda()) != W4A8_OK) return st;
+        dispatch_scan_kernel<<<1, kDispatchScanThreads, 0, s>>>(dcnt, C, E, bn, expert_offsets_out, mtile_off);
+        if ((st = last_cuda()) != W4A8_OK) return st;
+        dispatch_scatter_kernel<<<C, kDispatchThreads, 0, s>>>(topk_idx_out, T, E, topk, tpc, dcnt, perm, inv);
+    }
     if ((st = last_cuda()) != W4A8_OK) return st;
     // 3. quantize X straight into dispatch order
     if (!mark(2)) return W4A8_ERR_CUDA;

@@ -37,7 +37,8 @@ def _weights(K, N, seed, symmetric, outlier_p=0.0):
 
 @pytest.mark.parametrize("M,K", [(16, 512), (1, 4096), (37, 1408), (8, 7168), (300, 2048), (3, 8), (2, 8192),
                                  (1000, 1408), (129, 2056), (70, 4104),
-                                 (8192, 8), (8200, 512), (8193, 1408), (9000, 2048)])  # one warp per row
+                                 (9000, 2048),                                  # one CTA per row
+                                 (8192, 8), (8200, 512), (8193, 1408), (8192, 1536)])  # one warp per row
 def test_quant_act_bit_exact(m, M, K):
     inp = gen_linear(M, K, 64, seed=M + K, n_outliers=min(8, K // 2), outlier_scale=50.0)
     st = m.new_status("cuda")

@@ -227,3 +227,18 @@ def test_moe_asym_decode_config(m):
     res = run_layer(m, layer, inp, topk)
     tokens = np.random.default_rng(1).choice(T, 3, replace=False)
     check_layer(m, layer, inp, topk, res, tokens=tokens)
+
+
+@pytest.mark.parametrize("T,H,E,topk,I,g,sym,zipf", [
+    (3000, 128, 256, 8, 64, 64, False, 1.1),   # dispatch over 12 CTAs, skewed experts
+    (270000, 64, 16, 1, 64, 64, True, None),   # 528 CTAs of 512 tokens each
+])
+def test_moe_dispatch_many_tokens(m, T, H, E, topk, I, g, sym, zipf):
+    """Many tokens: the dispatch runs over several CTAs (count, scan, scatter);
+    offsets, permutation and inverse must equal the oracle's for every token,
+    and the expert path is checked on a sample."""
+    layer = Layer(m, seed=T % 1000 + E, E=E, H=H, I=I, group=g, sym=sym, w_outlier_p=0.001)
+    inp = gen_moe_activations(T, H, E, seed=5, zipf=zipf)
+    res = run_layer(m, layer, inp, topk)
+    tokens = np.random.default_rng(1).choice(T, 16, replace=False)
+    check_layer(m, layer, inp, topk, res, tokens=np.concatenate([[0, T - 1], tokens]))
