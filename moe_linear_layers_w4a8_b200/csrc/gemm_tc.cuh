@@ -749,7 +749,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         float* dst = tile_part + (long long)slot * (BN * 128) + r;
 #pragma unroll
                         for (int jj = 0; jj < CH; ++jj) dst[(hcol * CH + jj) * 128] = acc[jj];
-                        __threadfence();
+                        // Every epilogue thread's stores precede the barrier; the one
+                        // gpu-scope release store after it publishes them all.
                         named_bar_sync(3, kNumEpiWarps * 32);
                         if (ew == 0 && lane == 0) st_release_gpu_u64(flags + slot, p.epoch);
                     } else {
