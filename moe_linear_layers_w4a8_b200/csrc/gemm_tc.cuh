@@ -115,7 +115,7 @@ struct GemmCfg {
     static constexpr int NS_RAW = 512 / SLOT_COLS;
     static constexpr int NS = NS_RAW > 4 ? 4 : NS_RAW;
     // ring depths of the shared-memory streams (in chunks)
-    static constexpr int SPC = (BN == 16) ? 4 : (BN == 128 ? 2 : 3);
+    static constexpr int SPC = (BN <= 32) ? 4 : (BN == 128 ? 2 : 3);
     static constexpr int SAC = (SGA * ACT_TILE <= 16384) ? 3 : (BN == 128 ? 3 : 2);
     static constexpr int SWC = 4;
     static constexpr int A_COL0 = NS * S * BN;           // first TMEM column of the weight tiles
@@ -765,7 +765,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         named_bar_sync(3, kNumEpiWarps * 32);
                         const bool reduce = !*wc.abort;
                         if (reduce) {
-                            __threadfence();
+                            // the flags were read with acquire before the barrier
                             // slot order: own partial first, then slots 1, 2, ...
                             constexpr int JW = CH < 16 ? CH : 16;
 #pragma unroll
