@@ -170,6 +170,12 @@ W4A8_API w4a8_status w4a8_quant_act(const uint16_t* X, int M, int K, int ldx, in
  * Y       device bf16 [M][ldy], ldy >= N.
  * workspace / ws_bytes: device scratch of at least
  *         w4a8_gemm_workspace_size(M, w) bytes (may be NULL when that is 0).
+ *         Split-K keeps fp32 partial tiles and per-tile flags there.  The
+ *         flags carry a per-launch epoch, so the workspace needs no
+ *         initialisation and may be reused freely; the one exception: after a
+ *         launch that ended with W4A8_ERR_TIMEOUT, zero the workspace before
+ *         replaying a captured graph of that launch (a replay repeats the
+ *         epoch).  Calls that can overlap on the GPU need separate workspaces.
  * Errors: INVALID_ARG, FORMAT_MISMATCH (bad descriptor), WORKSPACE,
  *         UNSUPPORTED_SHAPE; TIMEOUT via dev_status.
  */
