@@ -272,3 +272,24 @@ def test_gemm_strided_output(m, M):
     assert Ys.stride(0) == N + 3
     assert np.array_equal(bits(Ys), bits(Yc))
     assert (big[:, N:] == -7.0).all()
+
+
+@pytest.mark.parametrize("M,K,N,g,sym", [(5, 16384, 384, 128, True), (3, 12288, 320, 64, False)])
+def test_gemm_long_k(m, M, K, N, g, sym):
+    """K beyond the activation-quantization kernel's limit (the GEMM takes any
+    K that is a multiple of 16 and of the group): q_x and s_x come from the
+    oracle's quantization, uploaded; 128 / 192 groups per tile, split-K."""
+    inp = gen_linear(M, K, N, seed=K + M, n_outliers=8, outlier_scale=50.0)
+    W = inp.W if sym else _weights(K, N, 9, False)
+    pw = m.w4a8_pack_weights(W.cuda(), g, sym)
+    codes, s, z, _ = O.quant_weights(W.numpy(), g, sym)
+    qo, so, _, _ = O.quant_act(bits(inp.X))
+    q = torch.from_numpy(qo).cuda()
+    sx = torch.from_numpy(so).cuda()
+    st = m.new_status("cuda")
+    Y, P = m.w4a8_gemm_debug_partials(q, sx, pw, status=st)
+    assert m.w4a8_get_device_status(st) == 0
+    Po = O.partials(qo, codes, None if sym else z, g)
+    assert np.array_equal(P.cpu().numpy(), Po)
+    Ye, A = O.scale_partials(Po, so, s)
+    check_bf16(bits(Y), Ye, A)
