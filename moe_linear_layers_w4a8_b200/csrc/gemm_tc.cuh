@@ -755,10 +755,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         if (ew == 0 && lane == 0) st_release_gpu_u64(flags + slot, p.epoch);
                     } else {
                         if (ew == 0) {
+                            // slots 1 .. nsl-1, 32 at a time (nsl exceeds 32 for
+                            // narrow N with long K)
                             bool got = true;
-                            if (lane >= 1 && lane < nsl) {
-                                got = spin_until_equal_u64(flags + lane, p.epoch, wc);
-                                if (got) st_release_gpu_u64(flags + lane, 0ull);  // consumed
+                            for (int f = 1 + lane; f < nsl && got; f += 32) {
+                                got = spin_until_equal_u64(flags + f, p.epoch, wc);
+                                if (got) st_release_gpu_u64(flags + f, 0ull);  // consumed
                             }
                             if (!__all_sync(0xFFFFFFFFu, got) && lane == 0) *wc.abort = 1;
                         }
