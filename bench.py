@@ -244,7 +244,9 @@ class MoEWorkload:
         self.T, self.H, self.E, self.topk, self.I = c["T"], c["H"], c["E"], c["topk"], c["I"]
         self.group, self.sym, self.zipf, self.wp = c["group"], c["symmetric"], c["zipf"], c["w_outlier_p"]
         self.dev = device
-        self.launches_per_step = 7
+        # route, dispatch (one kernel, or count / scan / scatter above 256 tokens), quantize X,
+        # gate_up, quantize h, down, combine
+        self.launches_per_step = 7 + (2 if self.T > 256 else 0)
 
     def _weight(self, e, which, device):
         from synth import gen_expert_weight
