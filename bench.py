@@ -2,23 +2,30 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload decode|prefill|moe_sym|moe_asym_decode|moe_asym_prefill]
-                    [--m M]
+                    [--m M] [--main-only] [--no-cpu-baseline]
 
-One "step" is one pass of the hot path over one batch of synthetic input:
-  decode / prefill:  per-token INT8 quantization of X, then the W4A8 GEMM;
-  moe_*:             the whole MoE layer (route, dispatch + quantize, grouped
-                     gate_up with SiLU*up, quantize h, grouped down, combine).
+One "step" is one pass of the hot path over one batch of synthetic input,
+through the public call a user makes:
+  decode / prefill:  w4a8_linear (per-token INT8 quantization of X, then the
+                     W4A8 GEMM launched to overlap it);
+  moe_*:             w4a8_moe_grouped_gemm (route, dispatch + quantize,
+                     grouped gate_up with SiLU*up, quantize h, grouped down,
+                     combine).
 The default workload is the decode-shaped linear (M=32, K=4096, N=14336,
 symmetric int4 group 128, 8 outlier channels x50), whose metric is the
-weight bytes streamed per second.
+weight bytes streamed per second; its figures form the contract line, and
+the metric's other parts (prefill TOPS, MoE tokens/s for the three MoE
+configurations) follow in a "workloads" object with the same figures each.
 
-Timing: W untimed warm-up steps, then exactly K steps, each bracketed by a
+Timing: W untimed warm-up steps, then exactly K steps, bracketed by a
 barrier + synchronize, timed with CUDA events on the launching stream (max
-over ranks).  The steps run as CUDA-graph replays; packed weights are
-rotated over enough copies that every step reads them from HBM, not L2.
-The dominant kernel's per-launch time is measured with CUDA events around
-its launches in the last graph replay of the timed region.  SM clocks and
-throttle reasons are sampled through NVML during the timed region.
+over ranks).  The timed steps are uninstrumented CUDA-graph replays of the
+public call; packed weights are rotated over enough copies that every decode
+step reads them from HBM, not L2 (the other workloads' operands exceed L2).
+The dominant kernel's per-launch time comes from separate, untimed
+instrumented replays (events around a chain of GEMM launches, or at the MoE
+layer's stage boundaries).  SM clocks and throttle reasons are sampled
+through NVML during the timed region.
 
 `e2e` repeats the metric through the public API call a user makes, with the
 step's input copied host->device from pinned memory and the result read back
@@ -162,17 +169,42 @@ class LinearWorkload:
         self.launches_per_step = 2  # quantization + GEMM (split-K is summed inside the GEMM)
 
     def step(self, i, ev=None):
+        # the public one-call layer: the GEMM's weight streaming overlaps the quantization
+        self.m.w4a8_linear(self.X, self.copies[i % len(self.copies)], out=self.Y, workspace=self.lws)
+
+    @property
+    def kernel_timing_note(self):
+        return (f"CUDA events around a graph of {self._chain} back-to-back w4a8_gemm launches "
+                f"(packed weights rotated, activations quantized once), mean per launch")
+
+    def kernel_time(self, torch):
+        """Per-launch duration of the GEMM: events around a chain of
+        back-to-back launches in a CUDA graph (separate, untimed replays)."""
         m = self.m
-        w = self.copies[i % len(self.copies)]
-        if ev is None:
-            # the public one-call layer: the GEMM's weight streaming overlaps the quantization
-            m.w4a8_linear(self.X, w, out=self.Y, workspace=self.lws)
-            return
-        # timing replay: the same two kernels as separate calls, events around the GEMM alone
         m.w4a8_quant_act(self.X, q_out=self.q, s_out=self.s)
-        ev[0].record()
-        m.w4a8_gemm(self.q, self.s, w, out=self.Y, workspace=self.ws)
-        ev[1].record()
+        n = self._chain = 64 if self.decode else 8
+
+        def chain(i, ev):
+            if ev:
+                ev[0].record()
+            for j in range(n):
+                w = self.copies[(i * n + j) % len(self.copies)]
+                m.w4a8_gemm(self.q, self.s, w, out=self.Y, workspace=self.ws)
+            if ev:
+                ev[1].record()
+        g, evs = capture(torch, chain, 3, with_events=2)
+        times = []
+        for _ in range(2):
+            g.replay()
+            torch.cuda.synchronize()
+            times += [e[0].elapsed_time(e[1]) / n for e in evs]
+        del g
+        return statistics.mean(times), None
+
+    def release(self):
+        for a in ("copies", "X", "q", "s", "Y", "ws", "lws", "X_dev2", "Y_pin", "X_pin"):
+            if hasattr(self, a):
+                delattr(self, a)
 
     # metric
     def units(self):
@@ -280,6 +312,23 @@ class MoEWorkload:
         self.m.w4a8_moe_grouped_gemm(self.X, self.L, self.topk, self.w1, self.w2, workspace=self.ws, out=self.out,
                                      stage_events=ev)
 
+    kernel_timing_note = ("CUDA events at the layer's stage boundaries (w4a8_moe_grouped_gemm_profiled) in a "
+                          "separate, untimed graph replay of 4 layer steps; mean per stage")
+
+    def kernel_time(self, torch):
+        g, evs = capture(torch, self.step, 4, with_events=8)
+        g.replay()
+        torch.cuda.synchronize()
+        stage_ms = {name: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs)
+                    for i, name in enumerate(self.STAGES)}
+        del g
+        return stage_ms["gate_up"], stage_ms
+
+    def release(self):
+        for a in ("w1", "w2", "ws", "out", "X", "L", "X2", "L2", "out_pin", "X_pin", "L_pin"):
+            if hasattr(self, a):
+                delattr(self, a)
+
     def units(self):
         return self.T / 1e6, "Mtokens/s", "tokens per second through the whole layer"
 
@@ -292,11 +341,11 @@ class MoEWorkload:
         ops = 2.0 * R * H * 2 * I
         if self.name == "moe_asym_decode":
             return dict(bound="hbm", per_launch=self.hit * w1_expert + act, unit="GB/s", scale=1e9,
-                        peak=peaks["hbm"], kernel="gate_up",
+                        peak=peaks["hbm"], kernel="gate_up", kernel_name="w4a8_gemm_tc_kernel (gate_up)",
                         peak_note=f"hbm_gbs ({peaks['source']}); gate_up launch bytes = experts hit ({self.hit}) "
                                   f"x (packed gate_up weights + scales + zero-points) + activations in/out")
         return dict(bound="tensor", per_launch=ops, unit="TOPS", scale=1e12, peak=2.0 * peaks["bf16_sus"],
-                    kernel="gate_up",
+                    kernel="gate_up", kernel_name="w4a8_gemm_tc_kernel (gate_up)",
                     peak_note=f"2 x bf16_tflops_sustained ({peaks['source']}); gate_up launch ops = 2*pairs*H*2I")
 
     def config(self):
@@ -419,68 +468,79 @@ def job_throughput(unit_scale, steps, world, t_ms):
     return unit_scale * steps * world / (t_ms / 1e3)
 
 
-def run_ours(args, world, rank, local):
-    import torch
-    import moe_linear_layers_w4a8_b200 as m
-    m.load_library()  # fails loudly without the CUDA library
-    peaks = measured_peaks()
-    wl = make_workload(args.workload, args.m)
-    wl.setup()
-    K, W = args.steps, args.warmup
-    unit_scale, unit, meaning = wl.units()
-    roof = wl.kernel_roofline(peaks)
+def upload_graph(torch, g):
+    """Uploads an instantiated CUDA graph to the device ahead of its first
+    replay (otherwise the first replay carries the upload); best effort."""
+    try:
+        from cuda.bindings import runtime as rt
+        rt.cudaGraphUpload(g.raw_cuda_graph_exec(), torch.cuda.current_stream().cuda_stream)
+        torch.cuda.synchronize()
+    except Exception:
+        pass
 
-    # graphs: warm-up graph (W steps), timed graph(s) of length Lg, the last
-    # replay with events around the dominant kernel.
-    Lg = max(1, min(K, 64 if args.workload in ("decode",) else 8))
+
+def timed_product_steps(torch, wl, K, W, world, local):
+    """W untimed warm-up steps, then exactly K steps of the public call
+    (uninstrumented CUDA-graph replays of `wl.step`), bracketed by a barrier +
+    synchronize and timed with CUDA events on the launching stream; returns
+    (max-over-ranks ms, clock summary)."""
+    Lg = max(1, min(K, 64 if wl.name == "decode" else 8))
     reps, rem = divmod(K, Lg)
     gw, _ = capture(torch, wl.step, max(W, 1))
     gt, _ = capture(torch, wl.step, Lg)
-    gev, evs = capture(torch, wl.step, Lg, with_events=2 if isinstance(wl, LinearWorkload) else 8)
     grem = capture(torch, wl.step, rem)[0] if rem else None
-
-    for _ in range(1 if W else 0):
-        gw.replay()
+    for g in (gt, grem):
+        if g is not None:
+            upload_graph(torch, g)
+    gw.replay()
     barrier_sync(torch, world)
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local)
     with sampler:
+        # An untimed ~50 us device spin ahead of the start event: the host
+        # enqueues the event and the graph launches meanwhile, so the timed
+        # region holds device work only, not the host's launch latency.
+        torch.cuda._sleep(100_000)
         start.record()
-        for r in range(reps):
-            (gev if r == reps - 1 else gt).replay()
+        for _ in range(reps):
+            gt.replay()
         if grem is not None:
             grem.replay()
         end.record()
         torch.cuda.synchronize()
     barrier_sync(torch, world)
-    t_ms = start.elapsed_time(end)
-    t_ms = max_over_ranks(torch, world, t_ms)
-    ms_per_step = t_ms / K
+    t_ms = max_over_ranks(torch, world, start.elapsed_time(end))
+    del gw, gt, grem
+    torch.cuda.synchronize()
+    return t_ms, sampler.summary()
+
+
+def measure(args, wl, K, W, peaks, world, rank, local, cpu_budget_s):
+    """Every figure of one workload: product-path throughput over K timed
+    steps, the dominant kernel against its roofline (from separate,
+    untimed instrumented replays), end to end from host buffers, and the
+    oracle on a bounded sample."""
+    import torch
+    wl.setup()
+    unit_scale, unit, meaning = wl.units()
+    roof = wl.kernel_roofline(peaks)
+    t_ms, clocks = timed_product_steps(torch, wl, K, W, world, local)
     value = job_throughput(unit_scale, K, world, t_ms)
 
-    # dominant-kernel time: events around its launches in the last replay
-    stage_ms = None
-    if reps > 0 and isinstance(wl, LinearWorkload):
-        k_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
-    elif reps > 0:
-        stage_ms = {name: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs)
-                    for i, name in enumerate(wl.STAGES)}
-        k_ms = stage_ms[roof["kernel"]]
-    else:
-        k_ms = ms_per_step
+    k_ms, stage_ms = wl.kernel_time(torch)
     achieved = roof["per_launch"] / roof["scale"] / (k_ms / 1e3)
     roofline = {"bound": roof["bound"], "achieved": round(achieved, 2), "peak": round(roof["peak"], 1),
                 "unit": roof["unit"], "frac": round(achieved / roof["peak"], 4),
-                "traffic": traffic_from_profiles(args.workload, roof), "kernel_ms": round(k_ms, 5),
-                "peak_source": roof["peak_note"], "algorithmic_per_launch": roof["per_launch"]}
-    if roof["bound"] == "hbm":
-        roofline["frac_note"] = "of measured" if peaks["source"] == "measured" else "of fallback"
+                "traffic": traffic_from_profiles(wl.name, roof), "kernel_ms": round(k_ms, 5),
+                "kernel": roof.get("kernel_name", "w4a8_gemm_tc_kernel"), "timing": wl.kernel_timing_note,
+                "peak_source": roof["peak_note"], "algorithmic_per_launch": roof["per_launch"],
+                "frac_note": "of measured" if peaks["source"] == "measured" else "of fallback"}
+    if stage_ms is not None:
+        roofline["stage_ms"] = {k: round(v, 5) for k, v in stage_ms.items()}
 
     # end to end through the public API with host buffers
-    del gw, gt, gev, grem
-    torch.cuda.synchronize()
     h2d, d2h = wl.e2e_setup()
-    Ke = max(1, min(K, 2000 if args.workload == "decode" else max(10, K // 4)))
+    Ke = max(1, min(K, 2000 if wl.name == "decode" else max(10, K // 4)))
     for i in range(min(W, 20)):
         wl.e2e_step(i)
     barrier_sync(torch, world)
@@ -493,25 +553,45 @@ def run_ours(args, world, rank, local):
     te = max_over_ranks(torch, world, s2.elapsed_time(e2))
     e2e_value = job_throughput(unit_scale, Ke, world, te)
 
-    line = {
-        "metric": METRIC, "value": round(value, 3), "unit": unit, "n_gpus": world, "steps": K, "warmup": W,
-        "ms_per_step": round(ms_per_step, 6), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+    out = {
+        "value": round(value, 3), "unit": unit, "steps": K, "warmup": W, "ms_per_step": round(t_ms / K, 6),
         "config": dict(wl.config(), quantity=meaning, parallelism=f"replicas x{world}",
                        global_batch=(getattr(wl, "M", None) or getattr(wl, "T", None)) * world),
         "roofline": roofline,
-        "e2e": {"value": round(e2e_value, 3), "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "steps": Ke},
+        "e2e": {"value": round(e2e_value, 3), "unit": unit, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": Ke},
         "gpu_launches": wl.launches_per_step * K,
-        "clocks": sampler.summary(),
+        "clocks": clocks,
     }
-    if stage_ms is not None:
-        roofline["stage_ms"] = {k: round(v, 5) for k, v in stage_ms.items()}
-        roofline["kernel"] = "w4a8_gemm_tc_kernel (gate_up)"
-    else:
-        roofline["kernel"] = "w4a8_gemm_tc_kernel"
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(wl, unit_scale, unit)
+        out["cpu_baseline"] = cpu_baseline(wl, unit_scale, unit, budget_s=cpu_budget_s)
+    wl.release()
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return out
+
+
+SECONDARY = ["prefill", "moe_sym", "moe_asym_decode", "moe_asym_prefill"]
+
+
+def run_ours(args, world, rank, local):
+    import torch
+    import moe_linear_layers_w4a8_b200 as m
+    m.load_library()  # fails loudly without the CUDA library
+    peaks = measured_peaks()
+    K, W = args.steps, args.warmup
+    main = measure(args, make_workload(args.workload, args.m), K, W, peaks, world, rank, local, 10.0)
+    line = {"metric": METRIC, "value": main["value"], "unit": main["unit"], "n_gpus": world, "steps": K,
+            "warmup": W, "ms_per_step": main["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "int8", "data": "synthetic"}
+    line.update({k: v for k, v in main.items() if k not in ("value", "unit", "steps", "warmup", "ms_per_step")})
+    if args.workload == "decode" and args.m is None and not args.main_only:
+        # the metric's other parts, each with its own figures, on the same box
+        line["workloads"] = {}
+        for name in SECONDARY:
+            Kw = min(K, DEFAULT_STEPS[name])
+            line["workloads"][name] = measure(args, make_workload(name, None), Kw, W, peaks, world, rank, local,
+                                              3.0)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -579,7 +659,7 @@ def _oracle_sample(wl):
         frac = wl.oracle_step_setup(n) if wl.decode else _linear_row_sample(wl, 16)
         return frac, (f"all {wl.N} output columns of the M={wl.M} decode step (weight quantization untimed)"
                       if wl.decode else f"16 of {wl.M} rows x all {wl.N} columns")
-    n = min(wl.T, 8 if wl.T > 64 else 4)
+    n = min(wl.T, 2 if wl.E >= 256 else (8 if wl.T > 64 else 4))
     return wl.oracle_step_setup(n), f"{n} of {wl.T} tokens through the whole layer"
 
 
@@ -666,6 +746,8 @@ def main(argv=None):
                     choices=["decode", "prefill", "moe_sym", "moe_asym_decode", "moe_asym_prefill"])
     ap.add_argument("--m", type=int, default=None, help="rows of the linear workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--main-only", action="store_true",
+                    help="measure only the main workload (no 'workloads' object)")
     args = ap.parse_args(argv)
     if args.steps is None:
         args.steps = DEFAULT_STEPS[args.workload]

@@ -321,6 +321,28 @@ typedef struct {
 W4A8_API w4a8_status w4a8_moe_workspace_layout(int T, int E, int topk, const w4a8_wdesc* w1,
                                       const w4a8_wdesc* w2, w4a8_moe_ws_layout* out);
 
+/*
+ * w4a8_moe_debug_partials — test-only variant of w4a8_moe_grouped_gemm
+ * (same arguments and results) whose grouped GEMMs also write the exact int32
+ * group partials of selected (token, slot) pairs as the tensor cores produced
+ * them ("Quantization: formats, error and the real execution path",
+ * "Correctness contract": partials are compared bit for bit).
+ * pair_slot  device int32 [T*topk]: for pair p = t*topk + j, the row of P1 / P2
+ *            that receives its partials, or -1 to skip the pair.
+ * P1         device int32 [S][H/group][2I]: gate_up partials, S = 1 + the
+ *            largest slot in pair_slot; column n < I is gate column n,
+ *            n >= I is up column n - I.
+ * P2         device int32 [S][I/group][H]: down partials.
+ * Rows of skipped pairs and unlisted slots are left untouched.
+ */
+W4A8_API w4a8_status w4a8_moe_debug_partials(
+    const uint16_t* X, const float* logits, int T, int E, int topk,
+    const uint8_t* w1_packed, const float* w1_s, const uint8_t* w1_z, const w4a8_wdesc* w1,
+    const uint8_t* w2_packed, const float* w2_s, const uint8_t* w2_z, const w4a8_wdesc* w2,
+    uint16_t* out, int32_t* topk_idx_out, float* topk_w_out, int32_t* expert_offsets_out,
+    void* workspace, size_t ws_bytes, int32_t* dev_status, void* stream,
+    const int32_t* pair_slot, int32_t* P1, int32_t* P2);
+
 /* --------------------------------------------------------------- status -- */
 
 /* Synchronizes `stream`, then reads the device status word (0 = W4A8_OK).

@@ -121,6 +121,8 @@ def load_library():
                                             ctypes.POINTER(WDesc), P, P, P, P, P, S, P, P]
         L.w4a8_moe_grouped_gemm_profiled.restype = st
         L.w4a8_moe_grouped_gemm_profiled.argtypes = L.w4a8_moe_grouped_gemm.argtypes + [P]
+        L.w4a8_moe_debug_partials.restype = st
+        L.w4a8_moe_debug_partials.argtypes = L.w4a8_moe_grouped_gemm.argtypes + [P, P, P]
         L.w4a8_get_device_status.restype = st
         L.w4a8_get_device_status.argtypes = [P, P]
         L.w4a8_selftest_bounded_wait.restype = st
@@ -329,11 +331,14 @@ def w4a8_moe_workspace_layout(T: int, E: int, topk: int, w1: PackedWeight, w2: P
 def w4a8_moe_grouped_gemm(X: torch.Tensor, logits: torch.Tensor, topk: int, w1: PackedWeight,
                           w2: PackedWeight, workspace: Optional[torch.Tensor] = None,
                           status: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
-                          stage_events=None):
+                          stage_events=None, debug_pair_slot: Optional[torch.Tensor] = None):
     """One MoE expert layer (route, dispatch, gate_up + SiLU*up, down, combine).
     Returns dict(out, topk_idx, topk_w, expert_offsets, workspace).
     stage_events: optional list of 8 torch.cuda.Event recorded at the stage
-    boundaries (see w4a8_moe_grouped_gemm_profiled)."""
+    boundaries (see w4a8_moe_grouped_gemm_profiled).
+    debug_pair_slot: optional int32 [T*topk] (test hook, w4a8_moe_debug_partials):
+    the result then also holds P1 int32 [S, H/g, 2I] and P2 int32 [S, I/g, H],
+    the exact group partials of the pairs with slot >= 0."""
     L = load_library()
     _need_cuda(X, logits)
     if X.dtype != torch.bfloat16 or logits.dtype != torch.float32:
@@ -358,13 +363,23 @@ def w4a8_moe_grouped_gemm(X: torch.Tensor, logits: torch.Tensor, topk: int, w1: 
             _p(w2.packed), _p(w2.s_w), _p(w2.z), ctypes.byref(w2.desc),
             _p(out), _p(idx), _p(pw), _p(offs), _p(workspace),
             workspace.numel() * workspace.element_size(), _p(status), _stream(dev)]
-    if stage_events is None:
+    extra = {}
+    if debug_pair_slot is not None:
+        S = int(debug_pair_slot.max().item()) + 1 if debug_pair_slot.numel() else 0
+        g = w1.desc.group
+        I = w1.N // 2
+        P1 = torch.zeros(max(S, 1), H // g, 2 * I, dtype=torch.int32, device=dev)
+        P2 = torch.zeros(max(S, 1), I // g, H, dtype=torch.int32, device=dev)
+        code = L.w4a8_moe_debug_partials(*args, _p(debug_pair_slot.to(dev, torch.int32).contiguous()),
+                                         _p(P1), _p(P2))
+        extra = dict(P1=P1, P2=P2)
+    elif stage_events is None:
         code = L.w4a8_moe_grouped_gemm(*args)
     else:
         evs = (ctypes.c_void_p * 8)(*[None if e is None else ctypes.c_void_p(e.cuda_event) for e in stage_events])
         code = L.w4a8_moe_grouped_gemm_profiled(*args, evs)
     _check(code, "w4a8_moe_grouped_gemm")
-    return dict(out=out, topk_idx=idx, topk_w=pw, expert_offsets=offs, workspace=workspace)
+    return dict(out=out, topk_idx=idx, topk_w=pw, expert_offsets=offs, workspace=workspace, **extra)
 
 
 def w4a8_selftest_bounded_wait(status: torch.Tensor, limit_ns: int = 1_000_000) -> None:

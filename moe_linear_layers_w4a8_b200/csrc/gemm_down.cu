@@ -3,9 +3,10 @@
 
 namespace w4a8 {
 
-int launch_gemm_down(int bn, int group, const GemmMaps& maps, const GemmParams& p, int grid,
+int launch_gemm_down(bool dbg, int bn, int group, const GemmMaps& maps, const GemmParams& p, int grid,
                       cudaStream_t stream) {
-    return launch_gemm_mode<kModeDown, false>(bn, group, maps, p, grid, stream);
+    return dbg ? launch_gemm_mode<kModeDown, true>(bn, group, maps, p, grid, stream)
+               : launch_gemm_mode<kModeDown, false>(bn, group, maps, p, grid, stream);
 }
 
 }  // namespace w4a8

@@ -80,9 +80,9 @@ int launch_gemm_plain(bool dbg, int bn, int group, const GemmMaps& maps, const G
                       cudaStream_t stream);
 int launch_gemm_splitk(bool dbg, int bn, int group, const GemmMaps& maps, const GemmParams& p, int grid,
                        cudaStream_t stream);
-int launch_gemm_gateup(int bn, int group, const GemmMaps& maps, const GemmParams& p, int grid,
+int launch_gemm_gateup(bool dbg, int bn, int group, const GemmMaps& maps, const GemmParams& p, int grid,
                        cudaStream_t stream);
-int launch_gemm_down(int bn, int group, const GemmMaps& maps, const GemmParams& p, int grid,
+int launch_gemm_down(bool dbg, int bn, int group, const GemmMaps& maps, const GemmParams& p, int grid,
                      cudaStream_t stream);
 
 }  // namespace w4a8

@@ -79,7 +79,9 @@ struct GemmParams {
     int slots;                   // split-K slots per tile
     unsigned long long* flags;   // split-K: [tiles][slots] "partial stored" flags (epoch values)
     unsigned long long epoch;    // this launch's epoch (nonzero)
-    int32_t* dbgP;               // optional [M][G][N] int32 partials (plain / split-K)
+    int32_t* dbgP;               // optional int32 partials [rows][G][N] (test hook)
+    const int32_t* dbg_map;      // grouped modes: slot of each (token, k) pair in dbgP, or -1
+    const int32_t* dbg_perm;     // grouped modes: dispatch row -> (token, k) pair
     int n_tiles;
     int m_tiles;                 // plain / split-K
     long long units_per_cta;     // plain / split-K (MoE derives it on device)
@@ -169,21 +171,28 @@ struct TileInfo {
 template <int BN, int MODE>
 __device__ __forceinline__ TileInfo decode_tile(const GemmParams& p, long long t) {
     TileInfo ti;
-    const int gm = (int)(t / p.n_tiles);
-    ti.nt = (int)(t % p.n_tiles);
     if constexpr (MODE == kModeGateUp || MODE == kModeDown) {
-        int lo = 0, hi = p.E - 1;  // last expert whose m-tile prefix is <= gm
+        // Tiles are ordered (expert, n-tile, m-tile): the m-tiles that share
+        // one weight tile of an expert are consecutive units, so they run back
+        // to back in one CTA and the repeated weight reads hit L2.
+        int lo = 0, hi = p.E - 1;  // last expert whose first tile index is <= t
         while (lo < hi) {
             const int mid = (lo + hi + 1) >> 1;
-            if (__ldg(p.mtile_off + mid) <= gm) lo = mid; else hi = mid - 1;
+            if ((long long)__ldg(p.mtile_off + mid) * p.n_tiles <= t) lo = mid; else hi = mid - 1;
         }
+        const int m0 = __ldg(p.mtile_off + lo);
+        const int mte = __ldg(p.mtile_off + lo + 1) - m0;
+        const long long local = t - (long long)m0 * p.n_tiles;
         ti.e = lo;
-        ti.mt = gm - __ldg(p.mtile_off + lo);
+        ti.nt = (int)(local / mte);
+        ti.mt = (int)(local % mte);
         const int r0 = __ldg(p.expert_off + lo);
         const int r1 = __ldg(p.expert_off + lo + 1);
         ti.row0 = r0 + ti.mt * BN;
         ti.rows_valid = min(BN, r1 - ti.row0);
     } else {
+        const int gm = (int)(t / p.n_tiles);
+        ti.nt = (int)(t % p.n_tiles);
         ti.e = 0;
         ti.mt = gm;
         ti.row0 = gm * BN;
@@ -695,8 +704,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                 const int f = b * BC + x, i = f / CH, c = f % CH;
                                 const int col = hcol * CH + c;
                                 if (i < ns && col < ti.rows_valid) {
-                                    const long long m = ti.row0 + col;
-                                    p.dbgP[(m * G + g0 + i) * p.N + n] = ((int32_t)(v[x] - kMagicBits)) >> pshift;
+                                    long long m = ti.row0 + col;
+                                    if constexpr (MODE == kModeGateUp || MODE == kModeDown)
+                                        m = p.dbg_map ? __ldg(p.dbg_map + __ldg(p.dbg_perm + m)) : -1;
+                                    if (m >= 0)
+                                        p.dbgP[(m * G + g0 + i) * p.N + n] = ((int32_t)(v[x] - kMagicBits)) >> pshift;
                                 }
                             }
                         }

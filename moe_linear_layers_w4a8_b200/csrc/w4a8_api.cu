@@ -115,8 +115,8 @@ w4a8_status launch_gemm(int mode, bool dbg, int bn, int group, const GemmMaps& m
     switch (mode) {
         case kModePlain: r = launch_gemm_plain(dbg, bn, group, maps, p, grid, stream); break;
         case kModeSplitK: r = launch_gemm_splitk(dbg, bn, group, maps, p, grid, stream); break;
-        case kModeGateUp: r = launch_gemm_gateup(bn, group, maps, p, grid, stream); break;
-        case kModeDown: r = launch_gemm_down(bn, group, maps, p, grid, stream); break;
+        case kModeGateUp: r = launch_gemm_gateup(dbg, bn, group, maps, p, grid, stream); break;
+        case kModeDown: r = launch_gemm_down(dbg, bn, group, maps, p, grid, stream); break;
         default: r = W4A8_ERR_UNSUPPORTED_SHAPE;
     }
     return static_cast<w4a8_status>(r);
@@ -473,13 +473,18 @@ w4a8_status w4a8_gemm_debug_partials(const int8_t* qx, const float* s_x, const u
     return gemm_impl(qx, s_x, packed, s_w, z, w, M, Y, ldy, P, workspace, ws_bytes, dev_status, stream);
 }
 
-w4a8_status w4a8_moe_grouped_gemm_profiled(const uint16_t* X, const float* logits, int T, int E, int topk,
-                                           const uint8_t* w1_packed, const float* w1_s, const uint8_t* w1_z,
-                                           const w4a8_wdesc* w1, const uint8_t* w2_packed, const float* w2_s,
-                                           const uint8_t* w2_z, const w4a8_wdesc* w2, uint16_t* out,
-                                           int32_t* topk_idx_out, float* topk_w_out, int32_t* expert_offsets_out,
-                                           void* workspace, size_t ws_bytes, int32_t* dev_status, void* stream,
-                                           void* const* stage_events) {
+}  // extern "C"
+
+namespace {
+
+// The MoE layer; with dbg_map, the grouped GEMMs also write the int32 group
+// partials of the flagged (token, k) pairs to P1 / P2 (test hook).
+w4a8_status moe_impl(const uint16_t* X, const float* logits, int T, int E, int topk, const uint8_t* w1_packed,
+                     const float* w1_s, const uint8_t* w1_z, const w4a8_wdesc* w1, const uint8_t* w2_packed,
+                     const float* w2_s, const uint8_t* w2_z, const w4a8_wdesc* w2, uint16_t* out,
+                     int32_t* topk_idx_out, float* topk_w_out, int32_t* expert_offsets_out, void* workspace,
+                     size_t ws_bytes, int32_t* dev_status, void* stream, void* const* stage_events,
+                     const int32_t* dbg_map, int32_t* P1, int32_t* P2) {
     w4a8_status st = check_moe(T, E, topk, w1, w2);
     if (st != W4A8_OK) return st;
     if (T == 0) return W4A8_OK;
@@ -576,7 +581,10 @@ w4a8_status w4a8_moe_grouped_gemm_profiled(const uint16_t* X, const float* logit
         p.I = I;
         p.status = dev_status;
         p.wait_ns = kDefaultWaitNs;
-        if ((st = launch_gemm(kModeGateUp, false, bn, group, maps, p, sms, s)) != W4A8_OK) return st;
+        p.dbgP = P1;
+        p.dbg_map = dbg_map;
+        p.dbg_perm = perm;
+        if ((st = launch_gemm(kModeGateUp, dbg_map != nullptr, bn, group, maps, p, sms, s)) != W4A8_OK) return st;
     }
     // 5. quantize h per (token, expert) row
     if (!mark(4)) return W4A8_ERR_CUDA;
@@ -607,7 +615,10 @@ w4a8_status w4a8_moe_grouped_gemm_profiled(const uint16_t* X, const float* logit
         p.E = E;
         p.status = dev_status;
         p.wait_ns = kDefaultWaitNs;
-        if ((st = launch_gemm(kModeDown, false, bn, group, maps, p, sms, s)) != W4A8_OK) return st;
+        p.dbgP = P2;
+        p.dbg_map = dbg_map;
+        p.dbg_perm = perm;
+        if ((st = launch_gemm(kModeDown, dbg_map != nullptr, bn, group, maps, p, sms, s)) != W4A8_OK) return st;
     }
     // 7. weighted combine
     if (!mark(6)) return W4A8_ERR_CUDA;
@@ -618,6 +629,35 @@ w4a8_status w4a8_moe_grouped_gemm_profiled(const uint16_t* X, const float* logit
     }
     if (!mark(7)) return W4A8_ERR_CUDA;
     return W4A8_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+w4a8_status w4a8_moe_grouped_gemm_profiled(const uint16_t* X, const float* logits, int T, int E, int topk,
+                                           const uint8_t* w1_packed, const float* w1_s, const uint8_t* w1_z,
+                                           const w4a8_wdesc* w1, const uint8_t* w2_packed, const float* w2_s,
+                                           const uint8_t* w2_z, const w4a8_wdesc* w2, uint16_t* out,
+                                           int32_t* topk_idx_out, float* topk_w_out, int32_t* expert_offsets_out,
+                                           void* workspace, size_t ws_bytes, int32_t* dev_status, void* stream,
+                                           void* const* stage_events) {
+    return moe_impl(X, logits, T, E, topk, w1_packed, w1_s, w1_z, w1, w2_packed, w2_s, w2_z, w2, out, topk_idx_out,
+                    topk_w_out, expert_offsets_out, workspace, ws_bytes, dev_status, stream, stage_events, nullptr,
+                    nullptr, nullptr);
+}
+
+w4a8_status w4a8_moe_debug_partials(const uint16_t* X, const float* logits, int T, int E, int topk,
+                                    const uint8_t* w1_packed, const float* w1_s, const uint8_t* w1_z,
+                                    const w4a8_wdesc* w1, const uint8_t* w2_packed, const float* w2_s,
+                                    const uint8_t* w2_z, const w4a8_wdesc* w2, uint16_t* out, int32_t* topk_idx_out,
+                                    float* topk_w_out, int32_t* expert_offsets_out, void* workspace,
+                                    size_t ws_bytes, int32_t* dev_status, void* stream, const int32_t* pair_slot,
+                                    int32_t* P1, int32_t* P2) {
+    if (!pair_slot || !P1 || !P2) return W4A8_ERR_INVALID_ARG;
+    return moe_impl(X, logits, T, E, topk, w1_packed, w1_s, w1_z, w1, w2_packed, w2_s, w2_z, w2, out, topk_idx_out,
+                    topk_w_out, expert_offsets_out, workspace, ws_bytes, dev_status, stream, nullptr, pair_slot, P1,
+                    P2);
 }
 
 w4a8_status w4a8_moe_grouped_gemm(const uint16_t* X, const float* logits, int T, int E, int topk,

@@ -1,8 +1,19 @@
 """Comparison helpers shared by the GPU parity tests (test code only)."""
+import os
+
 import numpy as np
 import torch
 
 import oracle as O
+
+# (test, what, elements that needed the fp32 accumulation bound, elements
+# checked) for every bf16 comparison; printed in the pytest terminal summary.
+FALLBACK_LOG = []
+
+
+def record_fallback(what: str, n_fallback: int, n_total: int):
+    test = os.environ.get("PYTEST_CURRENT_TEST", "?").split(" ")[0]
+    FALLBACK_LOG.append((test, what, int(n_fallback), int(n_total)))
 
 
 def bits(t: torch.Tensor) -> np.ndarray:
@@ -45,7 +56,9 @@ def check_bf16(y_bits: np.ndarray, Y_exact: np.ndarray, absY: np.ndarray, rel: f
             f"{what}: {int((~ok).sum())} / {ok.size} elements out of tolerance; first {i.tolist()}: "
             f"gpu={y[tuple(i[0])]!r} exact={Y_exact[tuple(i[0])]!r} ulps={d[tuple(i[0])]} "
             f"abs_terms={absY[tuple(i[0])]!r}")
-    return int(((d > 1) & fallback).sum())
+    n = int(((d > 1) & fallback).sum())
+    record_fallback(what, n, ok.size)
+    return n
 
 
 def to_dev(a: np.ndarray, dtype=None, device="cuda"):

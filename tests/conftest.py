@@ -38,3 +38,23 @@ def orc():
     import oracle
     oracle.build()
     return oracle
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """Reports, for every bf16 comparison of the run, how many elements were
+    accepted by the fp32 accumulation bound rather than the 1-ulp bound."""
+    try:
+        from tests._util import FALLBACK_LOG
+    except Exception:
+        return
+    if not FALLBACK_LOG:
+        return
+    tr = terminalreporter
+    tot_fb = sum(r[2] for r in FALLBACK_LOG)
+    tot = sum(r[3] for r in FALLBACK_LOG)
+    tr.section("bf16 comparisons: elements accepted by the fp32 accumulation bound")
+    tr.write_line(f"{len(FALLBACK_LOG)} comparisons, {tot} elements, {tot_fb} needed the fp32 bound "
+                  f"({tot_fb / max(tot, 1):.2e} of all)")
+    for test, what, nfb, n in FALLBACK_LOG:
+        if nfb:
+            tr.write_line(f"  {test} [{what}]: {nfb} / {n}")

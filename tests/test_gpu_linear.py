@@ -183,6 +183,25 @@ def test_gemm_decode_shapes_full(m, M):
     check_bf16(bits(Y), Ye, A)
 
 
+@pytest.mark.parametrize("M", [1, 8, 32])
+def test_linear_decode_shapes_against_oracle(m, M):
+    """The product path itself (w4a8_linear: quantization + the GEMM
+    instantiation without the debug write, launched as the bench launches it)
+    at the decode shapes, every output element against the oracle."""
+    K, N, g = 4096, 14336, 128
+    inp = gen_linear(M, K, N, seed=0, n_outliers=8, outlier_scale=50.0)
+    pw = m.w4a8_pack_weights(inp.W.cuda(), g, True)
+    st = m.new_status("cuda")
+    ws = torch.empty(m.w4a8_linear_workspace_size(M, pw), dtype=torch.uint8, device="cuda")
+    Y = m.w4a8_linear(inp.X.cuda(), pw, workspace=ws, status=st)
+    Y2 = m.w4a8_linear(inp.X.cuda(), pw, workspace=ws, status=st)  # the same workspace again
+    assert m.w4a8_get_device_status(st) == 0
+    codes, s, _, _ = O.quant_weights(inp.W.numpy(), g, True)
+    res = O.linear(bits(inp.X), codes, s, None, g)
+    check_bf16(bits(Y), res["Y"], res["absY"], what=f"w4a8_linear M={M}")
+    assert np.array_equal(bits(Y2), bits(Y))
+
+
 def test_gemm_prefill_shape_sampled_rows(m):
     # Prefill-shaped linear at full size (M=8192, K=4096, N=14336): the GPU
     # computes everything in the launch configuration the bench times; the

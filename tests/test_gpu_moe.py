@@ -17,7 +17,7 @@ import torch
 
 import oracle as O
 from synth import gen_moe_activations, gen_expert_weight
-from tests._util import bf16_ordinal, bf16_ulp, bits, check_bf16
+from tests._util import bf16_ordinal, bf16_ulp, bits, check_bf16, record_fallback
 
 pytestmark = pytest.mark.gpu
 
@@ -62,11 +62,32 @@ class Layer:
         return self._codes[key]
 
 
-def run_layer(m, layer, inp, topk):
+def pair_slots(T, topk, tokens):
+    """int32 [T*topk]: the partials row of every pair of the sampled tokens
+    (token tokens[i], slot j -> i*topk + j), -1 elsewhere."""
+    ps = torch.full((T * topk,), -1, dtype=torch.int32)
+    for i, t in enumerate(tokens):
+        for j in range(topk):
+            ps[int(t) * topk + j] = i * topk + j
+    return ps
+
+
+def run_layer(m, layer, inp, topk, tokens=None):
+    """Runs the layer; with `tokens`, through the debug entry that also returns
+    the exact int32 group partials of those tokens' pairs (P1, P2)."""
     st = m.new_status("cuda")
-    res = m.w4a8_moe_grouped_gemm(inp.X.cuda(), inp.logits.cuda(), topk, layer.w1, layer.w2, status=st)
+    T = inp.X.shape[0]
+    ps = None if tokens is None else pair_slots(T, topk, tokens).cuda()
+    res = m.w4a8_moe_grouped_gemm(inp.X.cuda(), inp.logits.cuda(), topk, layer.w1, layer.w2, status=st,
+                                  debug_pair_slot=ps)
     assert m.w4a8_get_device_status(st) == 0
     return res
+
+
+def sample_tokens(T, n, seed, extra=()):
+    """Sorted unique token indices: `extra` plus n seeded draws."""
+    t = np.random.default_rng(seed).choice(T, min(n, T), replace=False)
+    return np.asarray(sorted(set(int(x) for x in np.concatenate([np.asarray(extra, dtype=np.int64), t]))))
 
 
 def check_layer(m, layer, inp, topk, res, tokens=None):
@@ -93,10 +114,14 @@ def check_layer(m, layer, inp, topk, res, tokens=None):
     tokens = np.asarray(sorted(set(int(t) for t in tokens)))
     rows = np.array([inv[t * topk + j] for t in tokens for j in range(topk)])
     expert_of_row = np.searchsorted(off_o, rows, side="right") - 1
+    # partials row of each dispatch row (the debug entry's pair slots)
+    tok_pos = {int(t): i for i, t in enumerate(tokens)}
+    slot_of_row = np.array([tok_pos[int(perm[r]) // topk] * topk + int(perm[r]) % topk for r in rows])
+    P1 = res["P1"].cpu().numpy() if "P1" in res else None
+    P2 = res["P2"].cpu().numpy() if "P2" in res else None
 
     # quantized X in dispatch order
     qx_o, sx_o, _, _ = O.quant_act(bits(inp.X)[tokens])
-    tok_pos = {int(t): i for i, t in enumerate(tokens)}
     qx = _ws_view(ws, lay["qx"], R, torch.int8, H).cpu().numpy()
     sx = _ws_view(ws, lay["sx"], R, torch.float32).cpu().numpy()
     for r in rows:
@@ -109,9 +134,15 @@ def check_layer(m, layer, inp, topk, res, tokens=None):
     yd = _ws_view(ws, lay["yd"], R, torch.int16, H).cpu().numpy().view(np.uint16)
     n_fallback = 0
     for e in np.unique(expert_of_row):
-        rs = rows[expert_of_row == e]
+        sel = expert_of_row == e
+        rs = rows[sel]
         c1, s1, z1 = layer.codes(int(e), 0)
         c2, s2, z2 = layer.codes(int(e), 1)
+        # gate_up partials, bit for bit
+        if P1 is not None:
+            Po1 = O.partials(qx[rs], c1, z1, g)
+            Pg1 = P1[slot_of_row[sel]]
+            assert np.array_equal(Pg1, Po1), f"gate_up partials: {int((Pg1 != Po1).sum())} differ (expert {e})"
         # gate_up, then h = silu(gate) * up
         Hx, Ha, _ = O.expert_linear_rows(qx[rs], sx[rs], c1, s1, z1, g)
         h_exact = O.silu_mul(Hx)
@@ -125,10 +156,15 @@ def check_layer(m, layer, inp, topk, res, tokens=None):
         hv = O.bf16_to_f32(h[rs]).astype(np.float64)
         ok = (d <= 1) | (np.abs(hv - hx) <= bound)
         assert ok.all(), f"h: {int((~ok).sum())} elements out of tolerance (expert {e})"
+        record_fallback(f"h (expert {e})", int(((d > 1) & ok).sum()), d.size)
         # quantization of the GPU's h
         qh_o, sh_o, _, _ = O.quant_act(np.ascontiguousarray(h[rs]))
         assert np.array_equal(qh[rs], qh_o) and np.array_equal(sh[rs], sh_o)
-        # down
+        # down partials, bit for bit, then the bf16 expert rows
+        if P2 is not None:
+            Po2 = O.partials(qh[rs], c2, z2, g)
+            Pg2 = P2[slot_of_row[sel]]
+            assert np.array_equal(Pg2, Po2), f"down partials: {int((Pg2 != Po2).sum())} differ (expert {e})"
         Yx, Ya, _ = O.expert_linear_rows(qh[rs], sh[rs], c2, s2, z2, g)
         n_fallback += check_bf16(yd[rs], Yx, Ya, what=f"expert {e} down output")
 
@@ -179,7 +215,7 @@ SMALL = [
 def test_moe_small_stagewise(m, T, H, E, topk, I, g, sym, zipf):
     layer = Layer(m, seed=T + E, E=E, H=H, I=I, group=g, sym=sym, w_outlier_p=0.001)
     inp = gen_moe_activations(T, H, E, seed=T * 3 + E, zipf=zipf)
-    res = run_layer(m, layer, inp, topk)
+    res = run_layer(m, layer, inp, topk, tokens=np.arange(T))
     _, tokens = check_layer(m, layer, inp, topk, res)
     assert end_to_end_rms(layer, inp, topk, res, tokens[:16]) <= 1e-2
 
@@ -189,7 +225,7 @@ def test_moe_one_expert_takes_every_token(m):
     layer = Layer(m, seed=5, E=E, H=H, I=I, group=128, sym=True, w_outlier_p=0.0)
     inp = gen_moe_activations(T, H, E, seed=5)
     inp.logits[:, 3] += 100.0
-    res = run_layer(m, layer, inp, topk)
+    res = run_layer(m, layer, inp, topk, tokens=np.arange(T))
     offs = res["expert_offsets"].cpu().numpy()
     assert offs[3] == 0 and offs[4] == T
     check_layer(m, layer, inp, topk, res)
@@ -212,9 +248,9 @@ def test_moe_symmetric_config_sampled(m):
     T, H, E, topk, I = 4096, 2048, 64, 6, 1408
     layer = Layer(m, seed=0, E=E, H=H, I=I, group=128, sym=True, w_outlier_p=0.0)
     inp = gen_moe_activations(T, H, E, seed=0, zipf=None)
-    res = run_layer(m, layer, inp, topk)
-    tokens = np.random.default_rng(0).choice(T, 12, replace=False)
-    _, tokens = check_layer(m, layer, inp, topk, res, tokens=np.concatenate([[0, T - 1], tokens]))
+    tokens = sample_tokens(T, 12, 0, extra=[0, T - 1])
+    res = run_layer(m, layer, inp, topk, tokens=tokens)
+    _, tokens = check_layer(m, layer, inp, topk, res, tokens=tokens)
     assert end_to_end_rms(layer, inp, topk, res, tokens[:4]) <= 1e-2
 
 
@@ -224,8 +260,8 @@ def test_moe_asym_decode_config(m):
     T, H, E, topk, I = 64, 7168, 256, 8, 2048
     layer = Layer(m, seed=0, E=E, H=H, I=I, group=64, sym=False, w_outlier_p=0.001)
     inp = gen_moe_activations(T, H, E, seed=0, zipf=1.1)
-    res = run_layer(m, layer, inp, topk)
-    tokens = np.random.default_rng(1).choice(T, 3, replace=False)
+    tokens = sample_tokens(T, 3, 1)
+    res = run_layer(m, layer, inp, topk, tokens=tokens)
     check_layer(m, layer, inp, topk, res, tokens=tokens)
 
 
@@ -239,6 +275,21 @@ def test_moe_dispatch_many_tokens(m, T, H, E, topk, I, g, sym, zipf):
     and the expert path is checked on a sample."""
     layer = Layer(m, seed=T % 1000 + E, E=E, H=H, I=I, group=g, sym=sym, w_outlier_p=0.001)
     inp = gen_moe_activations(T, H, E, seed=5, zipf=zipf)
-    res = run_layer(m, layer, inp, topk)
-    tokens = np.random.default_rng(1).choice(T, 16, replace=False)
-    check_layer(m, layer, inp, topk, res, tokens=np.concatenate([[0, T - 1], tokens]))
+    tokens = sample_tokens(T, 16, 1, extra=[0, T - 1])
+    res = run_layer(m, layer, inp, topk, tokens=tokens)
+    check_layer(m, layer, inp, topk, res, tokens=tokens)
+
+
+def test_moe_asym_prefill_config(m):
+    """The asymmetric prefill configuration at full size: T=8192, hidden 7168,
+    256 experts, top-8 with Zipf(1.1) logits, I=2048, uint4 + zero-point,
+    group 64 (112 groups per gate_up tile, BN=128), 0.1% weight outliers x20.
+    Routing and dispatch are checked for every token; quantized X, the int32
+    partials of both grouped GEMMs, h, q_h and the expert rows for a seeded
+    sample of tokens; the combine for those tokens."""
+    T, H, E, topk, I = 8192, 7168, 256, 8, 2048
+    layer = Layer(m, seed=0, E=E, H=H, I=I, group=64, sym=False, w_outlier_p=0.001)
+    inp = gen_moe_activations(T, H, E, seed=0, zipf=1.1)
+    tokens = sample_tokens(T, 10, 2, extra=[0, 4095, T - 1])
+    res = run_layer(m, layer, inp, topk, tokens=tokens)
+    check_layer(m, layer, inp, topk, res, tokens=tokens)
