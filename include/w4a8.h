@@ -147,7 +147,8 @@ W4A8_API w4a8_status w4a8_pack_weights(const float* W, int K, int N, int group, 
  * rowsum   device int32 [M][K/group_for_rowsum] = per-group sum of codes
  *          ("Inference Quantization ch.1" §7, the term that multiplies a
  *          weight zero-point), or NULL with group_for_rowsum = 0.
- * Requires K % 8 == 0 and K <= 8192.
+ * Requires K % 8 == 0 and K <= 2^24 (rows longer than 8192 are read twice:
+ * once for the absmax, once for the codes).
  */
 W4A8_API w4a8_status w4a8_quant_act(const uint16_t* X, int M, int K, int ldx, int group_for_rowsum,
                            int8_t* qx, float* s_x, int32_t* rowsum,
@@ -197,7 +198,7 @@ W4A8_API size_t w4a8_linear_workspace_size(int M, const w4a8_wdesc* w);
  * only after the quantization kernel completed.  Results are identical to
  * w4a8_quant_act followed by w4a8_gemm.
  * X         device bf16 [M][ldx] (rows of K = w->K used), 16-byte aligned,
- *           ldx % 8 == 0, K <= 8192.
+ *           ldx % 8 == 0, K <= 2^24.
  * packed, s_w, z, w: as for w4a8_gemm.
  * Y         device bf16 [M][ldy], ldy >= N.
  * workspace device scratch of at least w4a8_linear_workspace_size(M, w)

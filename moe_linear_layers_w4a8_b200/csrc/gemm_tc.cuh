@@ -171,7 +171,24 @@ struct TileInfo {
 template <int BN, int MODE>
 __device__ __forceinline__ TileInfo decode_tile(const GemmParams& p, long long t) {
     TileInfo ti;
-    if constexpr (MODE == kModeGateUp || MODE == kModeDown) {
+    if constexpr (MODE == kModeGateUp) {
+        // Tiles are ordered (expert, m-tile, n-tile): the n-tiles of an m-tile
+        // run back to back, so the m-tiles whose last n-tile finishes in a CTA
+        // (and which that CTA then quantizes) are spread evenly over the CTAs.
+        const int gm = (int)(t / p.n_tiles);
+        ti.nt = (int)(t % p.n_tiles);
+        int lo = 0, hi = p.E - 1;  // last expert whose m-tile prefix is <= gm
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (__ldg(p.mtile_off + mid) <= gm) lo = mid; else hi = mid - 1;
+        }
+        ti.e = lo;
+        ti.mt = gm - __ldg(p.mtile_off + lo);
+        const int r0 = __ldg(p.expert_off + lo);
+        const int r1 = __ldg(p.expert_off + lo + 1);
+        ti.row0 = r0 + ti.mt * BN;
+        ti.rows_valid = min(BN, r1 - ti.row0);
+    } else if constexpr (MODE == kModeDown) {
         // Tiles are ordered (expert, n-tile, m-tile): the m-tiles that share
         // one weight tile of an expert are consecutive units, so they run back
         // to back in one CTA and the repeated weight reads hit L2.
@@ -330,6 +347,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // the other warps wait there (for the barriers and the TMEM allocation).
     if (warp == kWarpPack) {
         if (lane == 0) {
+            // A kernel launched after this one with programmatic stream
+            // serialization may be scheduled on SMs this grid frees; it waits
+            // for this grid's completion before touching anything it writes.
+            pdl_launch_dependents();
             for (int i = 0; i < C::SPC; ++i) {
                 mbar_init(&p_full[i], 1);
                 mbar_init(&p_empty[i], kUnpackWarps);

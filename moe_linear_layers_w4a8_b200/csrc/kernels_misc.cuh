@@ -30,9 +30,13 @@ __global__ void __launch_bounds__(kQuantThreads) quant_act_kernel(
     int32_t* __restrict__ rowsum, int group, const int32_t* __restrict__ dest, int dest_k,
     int32_t* status) {
     // A GEMM launched after this kernel with programmatic stream serialization
-    // may start its prologue and weight streaming now; it waits for this
-    // grid's completion before it reads q / s_x.
+    // may start its prologue and weight streaming now (it reads only packed
+    // weights and scales before it waits for this grid's completion).
+    // Launched the same way itself, this kernel may start while the preceding
+    // kernel is still running: X and the outputs are touched only after that
+    // kernel completed.
     pdl_launch_dependents();
+    pdl_wait_prerequisites();
     const int m = blockIdx.x;
     const int tid = threadIdx.x;
     const int nchunk = K >> 3;
@@ -79,6 +83,7 @@ __global__ void __launch_bounds__(kQuantThreads) quant_act_kernel(
     }
     const float s = __fdiv_rn(amax, 127.0f);
     const float d = (s > 0.0f) ? s : 1.0f;
+    const float r_d = __frcp_rn(d);  // for the exact quotient rounding (rne_quotient)
 
     const int nrows_out = dest ? dest_k : 1;
 #pragma unroll
@@ -91,7 +96,7 @@ __global__ void __launch_bounds__(kQuantThreads) quant_act_kernel(
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
             const uint32_t bits = (e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xFFFFu);
-            float t = rintf(__fdiv_rn(bf16_bits_to_f32(bits), d));
+            float t = rne_quotient(bf16_bits_to_f32(bits), d, r_d);
             t = fminf(fmaxf(t, -127.0f), 127.0f);
             const int qi = (int)t;
             csum += qi;
@@ -126,6 +131,88 @@ __global__ void __launch_bounds__(kQuantThreads) quant_act_kernel(
     }
 }
 
+// The same quantization for rows longer than quant_act_kernel holds in
+// registers (K > 8192): one CTA per row reads the row twice, first for the
+// absmax, then for the codes (the second pass mostly from L2).  Every value is
+// computed by the same operations, so codes, scales and code sums are those of
+// quant_act_kernel.
+__global__ void __launch_bounds__(kQuantThreads) quant_act_long_kernel(
+    const uint16_t* __restrict__ X, int K, int ldx, int8_t* __restrict__ q, float* __restrict__ s_x,
+    int32_t* __restrict__ rowsum, int group, int32_t* status) {
+    pdl_launch_dependents();
+    pdl_wait_prerequisites();
+    const int m = blockIdx.x;
+    const int tid = threadIdx.x;
+    const int nchunk = K >> 3;
+    const uint4* xr = reinterpret_cast<const uint4*>(X + (size_t)m * ldx);
+
+    float amax = 0.0f;
+    uint32_t bad = 0;
+    for (int c = tid; c < nchunk; c += kQuantThreads) {
+        const uint4 raw = __ldg(xr + c);
+        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+            const uint32_t lo = w[h] & 0xFFFFu, hi = w[h] >> 16;
+            bad |= ((lo & 0x7F80u) == 0x7F80u) | ((hi & 0x7F80u) == 0x7F80u);
+            amax = fmaxf(amax, fabsf(bf16_bits_to_f32(lo)));
+            amax = fmaxf(amax, fabsf(bf16_bits_to_f32(hi)));
+        }
+    }
+    __shared__ float red_max[kQuantThreads / 32];
+    __shared__ uint32_t red_bad[kQuantThreads / 32];
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
+        bad |= __shfl_xor_sync(0xFFFFFFFFu, bad, off);
+    }
+    if ((tid & 31) == 0) {
+        red_max[tid >> 5] = amax;
+        red_bad[tid >> 5] = bad;
+    }
+    __syncthreads();
+    amax = red_max[0];
+    bad = red_bad[0];
+#pragma unroll
+    for (int i = 1; i < kQuantThreads / 32; ++i) {
+        amax = fmaxf(amax, red_max[i]);
+        bad |= red_bad[i];
+    }
+    const float s = __fdiv_rn(amax, 127.0f);
+    const float d = (s > 0.0f) ? s : 1.0f;
+    const float r_d = __frcp_rn(d);  // for the exact quotient rounding (rne_quotient)
+
+    // all threads run the same number of iterations (the code-sum shuffles
+    // need every lane); chunks past the row end hold zeros
+    for (int c0 = 0; c0 < nchunk; c0 += kQuantThreads) {
+        const int c = c0 + tid;
+        const bool live = c < nchunk;
+        const uint4 raw = live ? __ldg(xr + c) : make_uint4(0, 0, 0, 0);
+        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+        uint32_t packed[2] = {0u, 0u};
+        int32_t csum = 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const uint32_t bits = (e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xFFFFu);
+            float t = rne_quotient(bf16_bits_to_f32(bits), d, r_d);
+            t = fminf(fmaxf(t, -127.0f), 127.0f);
+            const int qi = (int)t;
+            csum += qi;
+            packed[e >> 2] |= ((uint32_t)(qi & 0xFF)) << (8 * (e & 3));
+        }
+        if (live) *reinterpret_cast<uint2*>(q + (size_t)m * K + (size_t)c * 8) = make_uint2(packed[0], packed[1]);
+        if (rowsum) {
+            const int lanes = group >> 3;
+            for (int off = lanes >> 1; off > 0; off >>= 1) csum += __shfl_xor_sync(0xFFFFFFFFu, csum, off);
+            if (live && (c % lanes) == 0) rowsum[(size_t)m * (K / group) + c / lanes] = csum;
+        }
+    }
+    if (tid == 0) {
+        s_x[m] = s;
+        if (bad) report_status(status, kStatusNonfinite);
+    }
+}
+
 // The same quantization with one warp per row (8 rows per CTA): no block-wide
 // reduction, and many more rows in flight per SM, for launches with many rows
 // of at most 4096 elements.  Lane l holds chunks l, l + 32, ... of its row, so
@@ -138,6 +225,7 @@ __global__ void __launch_bounds__(32 * kQuantRowsPerCta) quant_act_rows_kernel(
     const uint16_t* __restrict__ X, int rows, int K, int ldx, int8_t* __restrict__ q, float* __restrict__ s_x,
     int32_t* __restrict__ rowsum, int group, const int32_t* __restrict__ dest, int dest_k, int32_t* status) {
     pdl_launch_dependents();
+    pdl_wait_prerequisites();
     const int lane = threadIdx.x & 31;
     const int m = blockIdx.x * kQuantRowsPerCta + (threadIdx.x >> 5);
     if (m >= rows) return;  // warp-uniform
@@ -171,6 +259,7 @@ __global__ void __launch_bounds__(32 * kQuantRowsPerCta) quant_act_rows_kernel(
     }
     const float s = __fdiv_rn(amax, 127.0f);
     const float d = (s > 0.0f) ? s : 1.0f;
+    const float r_d = __frcp_rn(d);  // for the exact quotient rounding (rne_quotient)
 
     const int nrows_out = dest ? dest_k : 1;
 #pragma unroll
@@ -183,7 +272,7 @@ __global__ void __launch_bounds__(32 * kQuantRowsPerCta) quant_act_rows_kernel(
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
             const uint32_t bits = (e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xFFFFu);
-            float t = rintf(__fdiv_rn(bf16_bits_to_f32(bits), d));
+            float t = rne_quotient(bf16_bits_to_f32(bits), d, r_d);
             t = fminf(fmaxf(t, -127.0f), 127.0f);
             const int qi = (int)t;
             csum += qi;

@@ -89,12 +89,9 @@ __host__ __device__ constexpr long long wait_cycles_for_ns(unsigned long long ns
     return (long long)(ns * 2ull);
 }
 
-// Waits for the phase of `bar` with the given parity to complete.  Returns
-// false (after recording W4A8_ERR_TIMEOUT = 5) once `limit_cycles` SM cycles
-// have passed, or when another wait of the CTA already gave up.  The SM
-// cycle counter is cheap to read, so the common path costs one try_wait.
-__device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
-    if (mbar_try_wait(bar, parity)) return true;
+// Slow path of wait_bounded: sleep-polls until the phase completes, the CTA
+// aborts or the limit runs out.
+__device__ __forceinline__ bool wait_bounded_slow(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
     const long long t0 = clock64();
     while (true) {
         if (mbar_try_wait_sleep(bar, parity, 100000u)) return true;  // sleeps <= ~0.1 ms
@@ -105,6 +102,27 @@ __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, con
             return false;
         }
     }
+}
+
+// Waits for the phase of `bar` with the given parity to complete.  Returns
+// false (after recording W4A8_ERR_TIMEOUT = 5) once `limit_cycles` SM cycles
+// have passed, or when another wait of the CTA already gave up.  The SM
+// cycle counter is cheap to read, so the common path costs one try_wait.
+__device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
+    if (mbar_try_wait(bar, parity)) return true;
+    return wait_bounded_slow(bar, parity, w);
+}
+
+// Round-half-to-even of the correctly rounded fp32 quotient x / d (the code
+// decision of the INT8 quantization), given r = the correctly rounded 1/d.
+// x * r is within 2^-22 |x/d| of the exact quotient, and so is the correctly
+// rounded quotient; for |x/d| <= 128 both lie on the same side of every
+// half-integer unless x * r is within 2^-15 of one.  Only then (about one
+// value in 10^4) is the quotient divided out exactly.
+__device__ __forceinline__ float rne_quotient(float x, float d, float r) {
+    const float t = x * r;
+    const float dist = fabsf(t - (floorf(t) + 0.5f));
+    return dist > 0x1p-14f ? rintf(t) : rintf(__fdiv_rn(x, d));
 }
 
 // Paired fp32 arithmetic (two independent IEEE round-to-nearest results per
@@ -360,6 +378,12 @@ template <int N>
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r);
 
 template <>
+__device__ __forceinline__ void tmem_st32<8>(uint32_t taddr, const uint32_t* r) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
+                 "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]));
+}
+
+template <>
 __device__ __forceinline__ void tmem_st32<16>(uint32_t taddr, const uint32_t* r) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
@@ -405,6 +429,18 @@ __device__ __forceinline__ void tmem_fill32<32>(uint32_t taddr, uint32_t v) {
         "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,"
         "%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(taddr),
         "r"(v));
+}
+
+// Per-warpgroup register budget (all 128 threads of the warpgroup execute
+// it): .dec hands registers back to the CTA's pool, .inc takes them (waiting
+// until enough are free).  N is a multiple of 8 in [24, 256].
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {

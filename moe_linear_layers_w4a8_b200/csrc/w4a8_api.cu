@@ -192,7 +192,7 @@ w4a8_status check_wdesc(const w4a8_wdesc* w) {
 
 w4a8_status gemm_impl(const int8_t* qx, const float* s_x, const uint8_t* packed, const float* s_w,
                       const uint8_t* z, const w4a8_wdesc* w, int M, uint16_t* Y, int ldy, int32_t* P,
-                      void* workspace, size_t ws_bytes, int32_t* dev_status, void* stream, bool pdl = false) {
+                      void* workspace, size_t ws_bytes, int32_t* dev_status, void* stream) {
     w4a8_status st = check_wdesc(w);
     if (st != W4A8_OK) return st;
     if (M < 0 || !Y || ldy < w->N) return W4A8_ERR_INVALID_ARG;
@@ -221,7 +221,10 @@ w4a8_status gemm_impl(const int8_t* qx, const float* s_x, const uint8_t* packed,
     p.Y = Y;
     p.ldy = ldy;
     p.vec16 = (aligned16(Y) && ldy % 8 == 0) ? 1 : 0;
-    p.pdl = pdl ? 1 : 0;
+    // Launched with programmatic stream serialization: the prologue and the
+    // weight stream may overlap the preceding kernel; activations, scales of
+    // the activations, Y and the workspace are touched only after it ended.
+    p.pdl = 1;
     p.partial = static_cast<float*>(workspace);
     p.slots = pl.slots;
     if (pl.splitk) {
@@ -238,8 +241,28 @@ w4a8_status gemm_impl(const int8_t* qx, const float* s_x, const uint8_t* packed,
     return launch_gemm(p.mode, P != nullptr, pl.bn, w->group, maps, p, pl.grid, s);
 }
 
+// Launches `kern` on `s`, with programmatic stream serialization when `pdl`
+// (the kernel may then start before the preceding kernel of the stream ends;
+// the quantization kernels wait for it before touching memory).
+template <typename... KArgs, typename... Args>
+w4a8_status launch_maybe_pdl(void (*kern)(KArgs...), unsigned grid, unsigned block, cudaStream_t s, bool pdl,
+                             Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    if (cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...) != cudaSuccess) return W4A8_ERR_CUDA;
+    return W4A8_OK;
+}
+
 w4a8_status launch_quant(const uint16_t* X, int rows, int K, int ldx, int8_t* q, float* s_x, int32_t* rowsum,
-                         int group, const int32_t* dest, int dest_k, int32_t* status, cudaStream_t s) {
+                         int group, const int32_t* dest, int dest_k, int32_t* status, cudaStream_t s,
+                         bool pdl = false) {
     if (rows == 0) return W4A8_OK;
     if (rows >= 8192 && K <= 1536) {
         // very many short rows (measured on B200: 24576 x 1408 80 -> 57 us;
@@ -249,22 +272,30 @@ w4a8_status launch_quant(const uint16_t* X, int rows, int K, int ldx, int8_t* q,
         const int cpl = need <= 1 ? 1 : need <= 2 ? 2 : need <= 4 ? 4 : need <= 6 ? 6 : need <= 8 ? 8 : need <= 12 ? 12 : 16;
         const unsigned blocks = (unsigned)((rows + kQuantRowsPerCta - 1) / kQuantRowsPerCta);
         const unsigned threads = 32 * kQuantRowsPerCta;
+        w4a8_status st = W4A8_ERR_UNSUPPORTED_SHAPE;
         switch (cpl) {
-#define W4A8_QROWS(n) case n: quant_act_rows_kernel<n><<<blocks, threads, 0, s>>>(X, rows, K, ldx, q, s_x, rowsum, group, dest, dest_k, status); break;
+#define W4A8_QROWS(n) case n: st = launch_maybe_pdl(quant_act_rows_kernel<n>, blocks, threads, s, pdl, X, rows, K, ldx, q, s_x, rowsum, group, dest, dest_k, status); break;
             W4A8_QROWS(1) W4A8_QROWS(2) W4A8_QROWS(4) W4A8_QROWS(6) W4A8_QROWS(8) W4A8_QROWS(12) W4A8_QROWS(16)
 #undef W4A8_QROWS
         }
-        return last_cuda();
+        return st != W4A8_OK ? st : last_cuda();
     }
     const int cpt = (K / 8 + kQuantThreads - 1) / kQuantThreads;
+    if (cpt > 4) {
+        // rows longer than 8192: two passes over the row (scatter form unused here)
+        if (dest) return W4A8_ERR_UNSUPPORTED_SHAPE;
+        const w4a8_status st = launch_maybe_pdl(quant_act_long_kernel, (unsigned)rows, kQuantThreads, s, pdl, X, K,
+                                                ldx, q, s_x, rowsum, group, status);
+        return st != W4A8_OK ? st : last_cuda();
+    }
+    w4a8_status st = W4A8_ERR_UNSUPPORTED_SHAPE;
     switch (cpt) {
-        case 1: quant_act_kernel<1><<<rows, kQuantThreads, 0, s>>>(X, K, ldx, q, s_x, rowsum, group, dest, dest_k, status); break;
-        case 2: quant_act_kernel<2><<<rows, kQuantThreads, 0, s>>>(X, K, ldx, q, s_x, rowsum, group, dest, dest_k, status); break;
-        case 3: quant_act_kernel<3><<<rows, kQuantThreads, 0, s>>>(X, K, ldx, q, s_x, rowsum, group, dest, dest_k, status); break;
-        case 4: quant_act_kernel<4><<<rows, kQuantThreads, 0, s>>>(X, K, ldx, q, s_x, rowsum, group, dest, dest_k, status); break;
+#define W4A8_QCTA(n) case n: st = launch_maybe_pdl(quant_act_kernel<n>, (unsigned)rows, kQuantThreads, s, pdl, X, K, ldx, q, s_x, rowsum, group, dest, dest_k, status); break;
+        W4A8_QCTA(1) W4A8_QCTA(2) W4A8_QCTA(3) W4A8_QCTA(4)
+#undef W4A8_QCTA
         default: return W4A8_ERR_UNSUPPORTED_SHAPE;
     }
-    return last_cuda();
+    return st != W4A8_OK ? st : last_cuda();
 }
 
 // ------------------------------------------------------------ MoE layout --
@@ -424,7 +455,7 @@ w4a8_status w4a8_quant_act(const uint16_t* X, int M, int K, int ldx, int group_f
     if (M == 0) return W4A8_OK;
     if (!X || !qx || !s_x) return W4A8_ERR_INVALID_ARG;
     if (K % 8 != 0 || ldx % 8 != 0 || !aligned16(X)) return W4A8_ERR_UNSUPPORTED_SHAPE;
-    if (K > 8192) return W4A8_ERR_UNSUPPORTED_SHAPE;
+    if (K > (1 << 24)) return W4A8_ERR_UNSUPPORTED_SHAPE;
     if (rowsum) {
         if (group_for_rowsum != 64 && group_for_rowsum != 128) return W4A8_ERR_INVALID_ARG;
         if (K % group_for_rowsum != 0) return W4A8_ERR_INVALID_ARG;
@@ -450,7 +481,7 @@ w4a8_status w4a8_linear(const uint16_t* X, int M, int ldx, const uint8_t* packed
     if (M < 0 || !Y || ldy < w->N) return W4A8_ERR_INVALID_ARG;
     if (M == 0) return W4A8_OK;
     if (!X || ldx < w->K) return W4A8_ERR_INVALID_ARG;
-    if (w->K % 8 != 0 || ldx % 8 != 0 || !aligned16(X) || w->K > 8192) return W4A8_ERR_UNSUPPORTED_SHAPE;
+    if (w->K % 8 != 0 || ldx % 8 != 0 || !aligned16(X) || w->K > (1 << 24)) return W4A8_ERR_UNSUPPORTED_SHAPE;
     const LinearLayout L = linear_layout(M, w);
     if (!workspace || ws_bytes < L.total || !aligned16(workspace)) return W4A8_ERR_WORKSPACE;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -463,7 +494,7 @@ w4a8_status w4a8_linear(const uint16_t* X, int M, int ldx, const uint8_t* packed
     // at entry: launched with programmatic stream serialization, its prologue
     // and weight streaming overlap the quantization.
     return gemm_impl(qx, sx, packed, s_w, z, w, M, Y, ldy, nullptr, ws + L.gemm, ws_bytes - L.gemm, dev_status,
-                     stream, true);
+                     stream);
 }
 
 w4a8_status w4a8_gemm_debug_partials(const int8_t* qx, const float* s_x, const uint8_t* packed, const float* s_w,

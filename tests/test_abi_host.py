@@ -137,7 +137,7 @@ def test_pack_rejects_bad_args(lib):
 def test_quant_rejects_bad_args(lib):
     assert lib.w4a8_quant_act(FAKE, 4, 512, 100, 0, FAKE, FAKE, None, None, None) == 1      # ldx < K
     assert lib.w4a8_quant_act(FAKE, 4, 500, 512, 0, FAKE, FAKE, None, None, None) == 2      # K % 8
-    assert lib.w4a8_quant_act(FAKE, 4, 16384, 16384, 0, FAKE, FAKE, None, None, None) == 2  # K too large
+    assert lib.w4a8_quant_act(FAKE, 4, (1 << 24) + 8, (1 << 24) + 8, 0, FAKE, FAKE, None, None, None) == 2  # K > 2^24
     assert lib.w4a8_quant_act(FAKE, 4, 512, 512, 96, FAKE, FAKE, FAKE, None, None) == 1     # bad group
     assert lib.w4a8_quant_act(FAKE, 4, 512, 512, 128, FAKE, FAKE, None, None, None) == 1    # group w/o rowsum
     assert lib.w4a8_quant_act(FAKE, 0, 512, 512, 0, FAKE, FAKE, None, None, None) == 0      # empty

@@ -295,20 +295,39 @@ def test_gemm_strided_output(m, M):
 
 @pytest.mark.parametrize("M,K,N,g,sym", [(5, 16384, 384, 128, True), (3, 12288, 320, 64, False)])
 def test_gemm_long_k(m, M, K, N, g, sym):
-    """K beyond the activation-quantization kernel's limit (the GEMM takes any
-    K that is a multiple of 16 and of the group): q_x and s_x come from the
-    oracle's quantization, uploaded; 128 / 192 groups per tile, split-K."""
+    """Long rows (K = 16384 / 12288: 128 / 192 groups per tile, split-K): the
+    quantization reads each row twice (absmax, then codes) and must give the
+    oracle's codes bit for bit; the one-call layer gives what quantization +
+    GEMM give; partials bit-exact."""
     inp = gen_linear(M, K, N, seed=K + M, n_outliers=8, outlier_scale=50.0)
     W = inp.W if sym else _weights(K, N, 9, False)
     pw = m.w4a8_pack_weights(W.cuda(), g, sym)
     codes, s, z, _ = O.quant_weights(W.numpy(), g, sym)
-    qo, so, _, _ = O.quant_act(bits(inp.X))
-    q = torch.from_numpy(qo).cuda()
-    sx = torch.from_numpy(so).cuda()
+    qo, so, rso, _ = O.quant_act(bits(inp.X), group=g)
     st = m.new_status("cuda")
+    q, sx, rs = m.w4a8_quant_act(inp.X.cuda(), group_for_rowsum=g, status=st)
+    assert np.array_equal(q.cpu().numpy(), qo)
+    assert np.array_equal(sx.cpu().numpy(), so)
+    assert np.array_equal(rs.cpu().numpy(), rso)
     Y, P = m.w4a8_gemm_debug_partials(q, sx, pw, status=st)
+    Y1 = m.w4a8_linear(inp.X.cuda(), pw, status=st)
     assert m.w4a8_get_device_status(st) == 0
     Po = O.partials(qo, codes, None if sym else z, g)
     assert np.array_equal(P.cpu().numpy(), Po)
     Ye, A = O.scale_partials(Po, so, s)
     check_bf16(bits(Y), Ye, A)
+    assert np.array_equal(bits(Y1), bits(Y))
+
+
+@pytest.mark.parametrize("M,K", [(3, 8200), (70, 16384), (2, 32768)])
+def test_quant_act_long_rows_bit_exact(m, M, K):
+    """Rows beyond 8192 elements (two passes over the row), with code sums."""
+    inp = gen_linear(M, K, 64, seed=M + K, n_outliers=8, outlier_scale=50.0)
+    st = m.new_status("cuda")
+    q, s, rs = m.w4a8_quant_act(inp.X.cuda(), group_for_rowsum=64 if K % 64 == 0 else 0, status=st)
+    qo, so, rso, bad = O.quant_act(bits(inp.X), group=64 if K % 64 == 0 else 0)
+    assert np.array_equal(q.cpu().numpy(), qo)
+    assert np.array_equal(s.cpu().numpy(), so)
+    if K % 64 == 0:
+        assert np.array_equal(rs.cpu().numpy(), rso)
+    assert m.w4a8_get_device_status(st) == 0 and not bad
