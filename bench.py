@@ -55,7 +55,7 @@ METRIC = "W4A8 GEMM TOPS (prefill) & weight GB/s (decode) vs B200 roofline; MoE 
 L2_BYTES = 126 * 1024 * 1024
 
 DEFAULT_STEPS = {"decode": 20000, "prefill": 1500, "moe_sym": 2000, "moe_asym_decode": 400,
-                 "moe_asym_prefill": 200}
+                 "moe_asym_prefill": 200, "w8a8_decode": 20000, "w8a8_prefill": 1500}
 
 
 # ---------------------------------------------------------------- peaks ---
@@ -140,7 +140,8 @@ class LinearWorkload:
     def __init__(self, name, M, K=4096, N=14336, group=128, device="cuda"):
         self.name, self.M, self.K, self.N, self.group = name, M, K, N, group
         self.dev = device
-        self.decode = name == "decode"
+        self.decode = name in ("decode", "w8a8_decode")
+        self.w8 = name.startswith("w8a8")  # per-channel INT8 weights (the W8A8 variant)
 
     def setup(self):
         import torch
@@ -150,31 +151,46 @@ class LinearWorkload:
         M, K, N, g = self.M, self.K, self.N, self.group
         inp = gen_linear(M, K, N, seed=0, n_outliers=8, outlier_scale=50.0)
         self.X_host = inp.X
-        pw = m.w4a8_pack_weights(inp.W.to(self.dev), g, True)
-        self.w_bytes = N * K // 2 + (K // g) * N * 4
+        if self.w8:
+            pw = m.w8a8_pack_weights(inp.W.to(self.dev))
+            self.w_bytes = N * K + N * 4
+        else:
+            pw = m.w4a8_pack_weights(inp.W.to(self.dev), g, True)
+            self.w_bytes = N * K // 2 + (K // g) * N * 4
         # enough weight copies that the weights of consecutive steps are not in L2
         self.copies = [pw]
         if self.decode:
             n = max(2, math.ceil(2 * L2_BYTES / self.w_bytes) + 1)
             for _ in range(n - 1):
-                self.copies.append(m.PackedWeight(pw.packed.clone(), pw.s_w.clone(), None, pw.desc.copy()))
+                if self.w8:
+                    self.copies.append(m.PackedW8(pw.q_w.clone(), pw.s_w.clone(), pw.desc.copy()))
+                else:
+                    self.copies.append(m.PackedWeight(pw.packed.clone(), pw.s_w.clone(), None, pw.desc.copy()))
         self.X = inp.X.to(self.dev)
         self.q = torch.empty(M, K, dtype=torch.int8, device=self.dev)
         self.s = torch.empty(M, dtype=torch.float32, device=self.dev)
         self.Y = torch.empty(M, N, dtype=torch.bfloat16, device=self.dev)
-        ws = m.w4a8_gemm_workspace_size(M, pw)
+        if self.w8:
+            ws = m.w8a8_gemm_workspace_size(M, pw)
+            lws = m.w8a8_linear_workspace_size(M, pw)
+            self._linear, self._gemm = m.w8a8_linear, m.w8a8_gemm
+        else:
+            ws = m.w4a8_gemm_workspace_size(M, pw)
+            lws = m.w4a8_linear_workspace_size(M, pw)
+            self._linear, self._gemm = m.w4a8_linear, m.w4a8_gemm
         self.ws = torch.empty(max(ws, 16), dtype=torch.uint8, device=self.dev)
-        self.lws = torch.empty(m.w4a8_linear_workspace_size(M, pw), dtype=torch.uint8, device=self.dev)
+        self.lws = torch.empty(lws, dtype=torch.uint8, device=self.dev)
         self.splitk = ws > 0
         self.launches_per_step = 2  # quantization + GEMM (split-K is summed inside the GEMM)
 
     def step(self, i, ev=None):
         # the public one-call layer: the GEMM's weight streaming overlaps the quantization
-        self.m.w4a8_linear(self.X, self.copies[i % len(self.copies)], out=self.Y, workspace=self.lws)
+        self._linear(self.X, self.copies[i % len(self.copies)], out=self.Y, workspace=self.lws)
 
     @property
     def kernel_timing_note(self):
-        return (f"CUDA events around a graph of {self._chain} back-to-back w4a8_gemm launches "
+        return (f"CUDA events around a graph of {self._chain} back-to-back "
+                f"{'w8a8_gemm' if self.w8 else 'w4a8_gemm'} launches "
                 f"(packed weights rotated, activations quantized once), mean per launch")
 
     def kernel_time(self, torch):
@@ -189,7 +205,7 @@ class LinearWorkload:
                 ev[0].record()
             for j in range(n):
                 w = self.copies[(i * n + j) % len(self.copies)]
-                m.w4a8_gemm(self.q, self.s, w, out=self.Y, workspace=self.ws)
+                self._gemm(self.q, self.s, w, out=self.Y, workspace=self.ws)
             if ev:
                 ev[1].record()
         g, evs = capture(torch, chain, 3, with_events=2)
@@ -215,7 +231,7 @@ class LinearWorkload:
     def kernel_roofline(self, peaks):
         M, K, N, g = self.M, self.K, self.N, self.group
         if self.decode:
-            alg = N * K // 2 + (K // g) * N * 4 + M * K + 4 * M + 2 * M * N
+            alg = self.w_bytes + M * K + 4 * M + 2 * M * N
             return dict(bound="hbm", per_launch=alg, unit="GB/s", scale=1e9, peak=peaks["hbm"],
                         peak_note=f"hbm_gbs ({peaks['source']})")
         ops = 2.0 * M * N * K
@@ -223,8 +239,9 @@ class LinearWorkload:
                     peak_note=f"2 x bf16_tflops_sustained ({peaks['source']}; int8/bf16 nominal ratio 2)")
 
     def config(self):
-        base = {"workload": f"{self.name} linear M={self.M} K={self.K} N={self.N} symmetric int4 g={self.group}",
-                "M": self.M, "K": self.K, "N": self.N, "group": self.group}
+        wfmt = "per-channel int8 weights (W8A8)" if self.w8 else f"symmetric int4 g={self.group}"
+        base = {"workload": f"{self.name} linear M={self.M} K={self.K} N={self.N} {wfmt}",
+                "M": self.M, "K": self.K, "N": self.N, "group": self.K if self.w8 else self.group}
         if not hasattr(self, "copies"):
             return base
         return dict(base, **{
@@ -243,7 +260,7 @@ class LinearWorkload:
 
     def e2e_step(self, i):
         self.X_dev2.copy_(self.X_pin, non_blocking=True)
-        Y = self.m.w4a8_linear(self.X_dev2, self.copies[i % len(self.copies)], out=self.Y, workspace=self.lws)
+        Y = self._linear(self.X_dev2, self.copies[i % len(self.copies)], out=self.Y, workspace=self.lws)
         self.Y_pin.copy_(Y, non_blocking=True)
 
     # CPU oracle on a bounded sample of the same workload
@@ -253,8 +270,13 @@ class LinearWorkload:
         import torch
         W = self._W_host()
         cols = np.sort(np.random.default_rng(0).choice(self.N, n_cols, replace=False))
-        codes, s, _, _ = O.quant_weights(W[:, cols].copy(), self.group, True)  # offline step, untimed
-        self._orc = (O, codes, s, self.X_host.view(torch.int16).numpy().view(np.uint16))
+        Xb = self.X_host.view(torch.int16).numpy().view(np.uint16)
+        if self.w8:
+            qw, sw, _ = O.quant_w8(W[:, cols].copy())  # offline step, untimed
+            self._orc = (O, qw, sw, Xb)
+        else:
+            codes, s, _, _ = O.quant_weights(W[:, cols].copy(), self.group, True)  # offline step, untimed
+            self._orc = (O, codes, s, Xb)
         return n_cols / self.N
 
     def _W_host(self):
@@ -263,7 +285,11 @@ class LinearWorkload:
 
     def oracle_step(self):
         O, codes, s, Xb = self._orc
-        O.linear(Xb, codes, s, None, self.group)
+        if self.w8:
+            qx, sx, _, _ = O.quant_act(Xb)
+            O.w8a8_exact(qx, sx, codes, s)
+        else:
+            O.linear(Xb, codes, s, None, self.group)
 
 
 class MoEWorkload:
@@ -401,8 +427,8 @@ class MoEWorkload:
 
 
 def make_workload(name, M):
-    if name in ("decode", "prefill"):
-        return LinearWorkload(name, M if M else (32 if name == "decode" else 8192))
+    if name in ("decode", "prefill", "w8a8_decode", "w8a8_prefill"):
+        return LinearWorkload(name, M if M else (32 if name.endswith("decode") else 8192))
     return MoEWorkload(name)
 
 
@@ -571,7 +597,7 @@ def measure(args, wl, K, W, peaks, world, rank, local, cpu_budget_s):
     return out
 
 
-SECONDARY = ["prefill", "moe_sym", "moe_asym_decode", "moe_asym_prefill"]
+SECONDARY = ["prefill", "moe_sym", "moe_asym_decode", "moe_asym_prefill", "w8a8_decode", "w8a8_prefill"]
 
 
 def run_ours(args, world, rank, local):
@@ -655,10 +681,10 @@ def cpu_baseline(wl, unit_scale, unit, budget_s=12.0):
 
 def _oracle_sample(wl):
     if isinstance(wl, LinearWorkload):
-        n = wl.N if wl.decode else 256
-        frac = wl.oracle_step_setup(n) if wl.decode else _linear_row_sample(wl, 16)
-        return frac, (f"all {wl.N} output columns of the M={wl.M} decode step (weight quantization untimed)"
-                      if wl.decode else f"16 of {wl.M} rows x all {wl.N} columns")
+        n = (1024 if wl.w8 else wl.N) if wl.decode else 256
+        frac = wl.oracle_step_setup(n) if wl.decode else _linear_row_sample(wl, 4 if wl.w8 else 16)
+        return frac, (f"{n} of {wl.N} output columns of the M={wl.M} decode step (weight quantization untimed)"
+                      if wl.decode else f"{4 if wl.w8 else 16} of {wl.M} rows x all {wl.N} columns")
     n = min(wl.T, 2 if wl.E >= 256 else (8 if wl.T > 64 else 4))
     return wl.oracle_step_setup(n), f"{n} of {wl.T} tokens through the whole layer"
 
@@ -668,8 +694,16 @@ def _linear_row_sample(wl, rows):
     import oracle as O
     import torch
     W = wl._W_host()
-    codes, s, _, _ = O.quant_weights(W, wl.group, True)
     Xb = wl.X_host.view(torch.int16).numpy().view(np.uint16)[:rows].copy()
+    if getattr(wl, "w8", False):
+        qw, sw, _ = O.quant_w8(W)
+
+        def step():
+            qx, sx, _, _ = O.quant_act(Xb)
+            O.w8a8_exact(qx, sx, qw, sw)
+        wl.oracle_step = step
+        return rows / wl.M
+    codes, s, _, _ = O.quant_weights(W, wl.group, True)
 
     def step():
         O.linear(Xb, codes, s, None, wl.group)
@@ -743,7 +777,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="decode",
-                    choices=["decode", "prefill", "moe_sym", "moe_asym_decode", "moe_asym_prefill"])
+                    choices=["decode", "prefill", "moe_sym", "moe_asym_decode", "moe_asym_prefill", "w8a8_decode",
+                             "w8a8_prefill"])
     ap.add_argument("--m", type=int, default=None, help="rows of the linear workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--main-only", action="store_true",

@@ -259,6 +259,52 @@ W4A8_API w4a8_status w4a8_gemm_static_scratch(const int8_t* qx, const float* s_x
                                      const w4a8_wdesc* w, int M, uint16_t* Y, int ldy,
                                      int32_t* dev_status, void* stream);
 
+/* ------------------------------------------------------------- W8A8 ---- */
+
+/*
+ * The W8A8 variant of the Linear layer ("Inference Quantization ch.1" §4, the
+ * INT8 ideal path, with §8.2 per-channel weight scales and §8.3 per-token
+ * activation scales):
+ *   s_w[n]   = max_k |W[k,n]| / 127,  q_w = clamp(rne(W / s_w), -127, 127)
+ *   acc[m,n] = sum_k q_x[m,k] q_w[k,n]                   (exact int32)
+ *   Y[m,n]   = s_x[m] * (s_w[n] * acc[m,n])              (fp32, bf16 output)
+ * q_x / s_x are w4a8_quant_act's.  Same kernel structure as w4a8_gemm without
+ * the 4-bit unpack and without per-group rescaling: the int32 accumulator
+ * spans all of K and the epilogue runs once per tile.
+ * Descriptor: bits = 8, symmetric = 1, group = K (one scale per column),
+ * layout_version = W4A8_LAYOUT_VERSION; the w4a8_* calls reject it.
+ * Weight layout: q_w int8 [N][K] row-major (k contiguous), s_w fp32 [N].
+ * Limits: K % 128 == 0, K <= 2^17 (so |acc| < 2^31), N % 16 == 0.
+ */
+
+/* w8a8_pack_weights — offline per-channel INT8 quantization of W fp32 [K][N]
+ * (device, row-major) into q_w / s_w as above; a zero column gives s_w = 0 and
+ * codes 0.  out (host) is filled on success.  Errors: INVALID_ARG (null
+ * pointers, K % 128, N % 16, q_w not 16-byte aligned); NONFINITE via
+ * dev_status. */
+W4A8_API w4a8_status w8a8_pack_weights(const float* W, int K, int N, int8_t* q_w, float* s_w, w4a8_wdesc* out,
+                                       int32_t* dev_status, void* stream);
+
+/* Workspace bytes w8a8_gemm needs for M rows (split-K int32 partial tiles and
+ * their flags; 0 when none). */
+W4A8_API size_t w8a8_gemm_workspace_size(int M, const w4a8_wdesc* w);
+
+/* w8a8_gemm — Y = W8A8(q_x, q_w).  qx int8 [M][K] and q_w 16-byte aligned;
+ * Y bf16 [M][ldy].  Workspace rules as for w4a8_gemm (split-K partials are
+ * int32, so their sum is exact in any order).  Errors as w4a8_gemm. */
+W4A8_API w4a8_status w8a8_gemm(const int8_t* qx, const float* s_x, const int8_t* q_w, const float* s_w,
+                               const w4a8_wdesc* w, int M, uint16_t* Y, int ldy, void* workspace, size_t ws_bytes,
+                               int32_t* dev_status, void* stream);
+
+/* Workspace bytes w8a8_linear needs for M rows (q_x, s_x, the GEMM's). */
+W4A8_API size_t w8a8_linear_workspace_size(int M, const w4a8_wdesc* w);
+
+/* w8a8_linear — per-token INT8 quantization of X bf16 [M][ldx] followed by
+ * w8a8_gemm, in one call (results identical to the two calls). */
+W4A8_API w4a8_status w8a8_linear(const uint16_t* X, int M, int ldx, const int8_t* q_w, const float* s_w,
+                                 const w4a8_wdesc* w, uint16_t* Y, int ldy, void* workspace, size_t ws_bytes,
+                                 int32_t* dev_status, void* stream);
+
 /*
  * w4a8_moe_grouped_gemm — one MoE expert layer, following "Kimi 2.7 MoE,
  * 4-bit storage to INT8" §4.1-4.4:

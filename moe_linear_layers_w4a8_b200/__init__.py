@@ -22,7 +22,8 @@ __all__ = [
     "w4a8_gemm_debug_partials", "w4a8_gemm_static_scratch", "w4a8_moe_grouped_gemm", "w4a8_moe_workspace_layout",
     "w4a8_gemm_workspace_size", "w4a8_moe_workspace_size", "w4a8_get_device_status",
     "w4a8_status_string", "w4a8_selftest_bounded_wait", "w4a8_linear", "w4a8_linear_workspace_size", "LAYOUT_VERSION",
-    "STATUS",
+    "STATUS", "PackedW8", "w8a8_pack_weights", "w8a8_gemm", "w8a8_gemm_workspace_size", "w8a8_linear",
+    "w8a8_linear_workspace_size",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -123,6 +124,16 @@ def load_library():
         L.w4a8_moe_grouped_gemm_profiled.argtypes = L.w4a8_moe_grouped_gemm.argtypes + [P]
         L.w4a8_moe_debug_partials.restype = st
         L.w4a8_moe_debug_partials.argtypes = L.w4a8_moe_grouped_gemm.argtypes + [P, P, P]
+        L.w8a8_pack_weights.restype = st
+        L.w8a8_pack_weights.argtypes = [P, I, I, P, P, ctypes.POINTER(WDesc), P, P]
+        L.w8a8_gemm_workspace_size.restype = S
+        L.w8a8_gemm_workspace_size.argtypes = [I, ctypes.POINTER(WDesc)]
+        L.w8a8_gemm.restype = st
+        L.w8a8_gemm.argtypes = [P, P, P, P, ctypes.POINTER(WDesc), I, P, I, P, S, P, P]
+        L.w8a8_linear_workspace_size.restype = S
+        L.w8a8_linear_workspace_size.argtypes = [I, ctypes.POINTER(WDesc)]
+        L.w8a8_linear.restype = st
+        L.w8a8_linear.argtypes = [P, I, I, P, P, ctypes.POINTER(WDesc), P, I, P, S, P, P]
         L.w4a8_get_device_status.restype = st
         L.w4a8_get_device_status.argtypes = [P, P]
         L.w4a8_selftest_bounded_wait.restype = st
@@ -385,3 +396,82 @@ def w4a8_moe_grouped_gemm(X: torch.Tensor, logits: torch.Tensor, topk: int, w1: 
 def w4a8_selftest_bounded_wait(status: torch.Tensor, limit_ns: int = 1_000_000) -> None:
     code = load_library().w4a8_selftest_bounded_wait(_p(status), int(limit_ns), _stream(status.device))
     _check(code, "w4a8_selftest_bounded_wait")
+
+
+# ------------------------------------------------------------------ W8A8 ---
+
+@dataclasses.dataclass
+class PackedW8:
+    """Per-channel INT8 weight of the W8A8 path: q_w int8 [N, K], s_w fp32 [N]."""
+    q_w: torch.Tensor
+    s_w: torch.Tensor
+    desc: WDesc
+
+    @property
+    def K(self):
+        return self.desc.K
+
+    @property
+    def N(self):
+        return self.desc.N
+
+
+def w8a8_pack_weights(W: torch.Tensor, status: Optional[torch.Tensor] = None) -> PackedW8:
+    """Per-channel INT8 quantization of W fp32 [K, N] (device)."""
+    L = load_library()
+    _need_cuda(W)
+    if W.dtype != torch.float32 or W.dim() != 2:
+        raise W4A8Error(1, "W must be fp32 [K, N]")
+    W = W.contiguous()
+    K, N = W.shape
+    q = torch.empty(N, K, dtype=torch.int8, device=W.device)
+    s = torch.empty(N, dtype=torch.float32, device=W.device)
+    d = WDesc()
+    _check(L.w8a8_pack_weights(_p(W), K, N, _p(q), _p(s), ctypes.byref(d), _p(status), _stream(W.device)),
+           "w8a8_pack_weights")
+    return PackedW8(q_w=q, s_w=s, desc=d)
+
+
+def w8a8_gemm_workspace_size(M: int, w: PackedW8) -> int:
+    return int(load_library().w8a8_gemm_workspace_size(int(M), ctypes.byref(w.desc)))
+
+
+def w8a8_gemm(qx: torch.Tensor, s_x: torch.Tensor, w: PackedW8, out: Optional[torch.Tensor] = None,
+              workspace: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Y bf16 [M, N] = W8A8(qx, w)."""
+    L = load_library()
+    _need_cuda(qx, s_x)
+    if qx.dtype != torch.int8 or qx.dim() != 2 or not qx.is_contiguous():
+        raise W4A8Error(1, "qx must be contiguous int8 [M, K]")
+    M = qx.shape[0]
+    if out is None:
+        out = torch.empty(M, w.N, dtype=torch.bfloat16, device=qx.device)
+    need = w8a8_gemm_workspace_size(M, w)
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=qx.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(L.w8a8_gemm(_p(qx), _p(s_x), _p(w.q_w), _p(w.s_w), ctypes.byref(w.desc), M, _p(out), out.stride(0),
+                       _p(workspace), ws_bytes, _p(status), _stream(qx.device)), "w8a8_gemm")
+    return out
+
+
+def w8a8_linear_workspace_size(M: int, w: PackedW8) -> int:
+    return int(load_library().w8a8_linear_workspace_size(int(M), ctypes.byref(w.desc)))
+
+
+def w8a8_linear(X: torch.Tensor, w: PackedW8, out=None, workspace=None, status=None) -> torch.Tensor:
+    """Y bf16 [M, N] = the W8A8 Linear layer on X bf16 [M, K] (quantization + GEMM)."""
+    L = load_library()
+    _need_cuda(X)
+    if X.dtype != torch.bfloat16 or X.dim() != 2 or X.stride(1) != 1:
+        raise W4A8Error(1, "X must be bf16 [M, K] with unit column stride")
+    M = X.shape[0]
+    if out is None:
+        out = torch.empty(M, w.N, dtype=torch.bfloat16, device=X.device)
+    need = w8a8_linear_workspace_size(M, w)
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=X.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(L.w8a8_linear(_p(X), M, X.stride(0), _p(w.q_w), _p(w.s_w), ctypes.byref(w.desc), _p(out), out.stride(0),
+                         _p(workspace), ws_bytes, _p(status), _stream(X.device)), "w8a8_linear")
+    return out

@@ -152,16 +152,6 @@ struct GemmCfg {
     static_assert(SMEM <= 227 * 1024, "shared memory");
 };
 
-struct Ring {
-    uint32_t idx = 0, phase = 0;
-    __device__ __forceinline__ void next(uint32_t n) {
-        if (++idx == n) {
-            idx = 0;
-            phase ^= 1u;
-        }
-    }
-};
-
 struct TileInfo {
     int e, mt, nt;
     int row0;        // first activation row of the tile
@@ -265,15 +255,6 @@ __device__ __forceinline__ Segment segment_at(long long u, long long u1, int G) 
     return sg;
 }
 
-// Steps back `n` uses of a ring (for the exit drains).
-__device__ __forceinline__ void ring_back(Ring& r, int n) {
-    if (r.idx == 0) {
-        r.idx = n - 1;
-        r.phase ^= 1u;
-    } else {
-        --r.idx;
-    }
-}
 
 // s_x of the tile's activation rows col0 .. col0 + JW - 1, all loads issued
 // back to back (indices clamped into the tile's valid rows; the values of

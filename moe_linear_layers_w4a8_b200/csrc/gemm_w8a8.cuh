@@ -325,3 +325,12 @@ __global__ void __launch_bounds__(kW8Threads, 1)
 }
 
 }  // namespace w4a8
+
+namespace w4a8 {
+
+// Launches the W8A8 kernel for a tile width BN in {16, 32, 64, 128, 256}
+// (defined in gemm_w8a8.cu).  Status codes as in w4a8.h.
+int launch_w8a8(int bn, bool split, const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, const W8Params& p,
+                int grid, cudaStream_t stream);
+
+}  // namespace w4a8

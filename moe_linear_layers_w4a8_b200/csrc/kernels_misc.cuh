@@ -653,6 +653,43 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
     *reinterpret_cast<uint4*>(out + (size_t)t * H + (size_t)c * 8) = make_uint4(o[0], o[1], o[2], o[3]);
 }
 
+// ---------------------------------------------------------------------------
+// Offline per-channel INT8 weight quantization for the W8A8 path
+// ("Inference Quantization ch.1" §2 worked example and §8.2 per-channel
+// scales): s_w[n] = max_k |W[k,n]| / 127, q = clamp(rne(W / s_w), -127, 127),
+// s_w == 0 -> divisor 1.  Output q_w[n][k] (k contiguous: the GEMM's weight
+// tile is one 2-D TMA box).  One thread per output column n (coalesced reads
+// of W across the warp); each thread writes its row 16 codes at a time.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(128) pack_w8_kernel(const float* __restrict__ W, int K, int N,
+                                                      int8_t* __restrict__ q_w, float* __restrict__ s_w,
+                                                      int32_t* status) {
+    const int n = blockIdx.x * blockDim.x + threadIdx.x;
+    if (n >= N) return;
+    float amax = 0.0f;
+    bool bad = false;
+    for (int k = 0; k < K; ++k) {
+        const float w = __ldg(W + (size_t)k * N + n);
+        bad |= !isfinite(w);
+        amax = fmaxf(amax, fabsf(w));
+    }
+    const float s = __fdiv_rn(amax, 127.0f);
+    const float d = (s > 0.0f) ? s : 1.0f;
+    int8_t* row = q_w + (size_t)n * K;
+    for (int k0 = 0; k0 < K; k0 += 16) {
+        uint32_t words[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+        for (int b = 0; b < 16; ++b) {
+            float t = rintf(__fdiv_rn(__ldg(W + (size_t)(k0 + b) * N + n), d));
+            t = fminf(fmaxf(t, -127.0f), 127.0f);
+            words[b >> 2] |= ((uint32_t)((int)t & 0xFF)) << (8 * (b & 3));
+        }
+        *reinterpret_cast<uint4*>(row + k0) = make_uint4(words[0], words[1], words[2], words[3]);
+    }
+    s_w[n] = s;
+    if (bad) report_status(status, kStatusNonfinite);
+}
+
 // Test hook: one warp waits on a barrier nobody arrives on.
 __global__ void bounded_wait_selftest_kernel(int32_t* status, unsigned long long limit_ns) {
     __shared__ __align__(8) uint64_t bar;

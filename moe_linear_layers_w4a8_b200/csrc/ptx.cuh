@@ -475,4 +475,25 @@ __device__ __forceinline__ bool warp_wait_bounded(uint64_t* bar, uint32_t parity
     return __all_sync(0xFFFFFFFFu, ok) != 0;
 }
 
+// Position in a ring of n stages and the parity of its current pass.
+struct Ring {
+    uint32_t idx = 0, phase = 0;
+    __device__ __forceinline__ void next(uint32_t n) {
+        if (++idx == n) {
+            idx = 0;
+            phase ^= 1u;
+        }
+    }
+};
+
+// Steps back `n` uses of a ring (for the exit drains).
+__device__ __forceinline__ void ring_back(Ring& r, int n) {
+    if (r.idx == 0) {
+        r.idx = n - 1;
+        r.phase ^= 1u;
+    } else {
+        --r.idx;
+    }
+}
+
 }  // namespace w4a8

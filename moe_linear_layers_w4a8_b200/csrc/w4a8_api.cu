@@ -16,6 +16,7 @@
 #include "w4a8.h"
 #include "gemm_launch.cuh"
 #include "kernels_misc.cuh"
+#include "gemm_w8a8.cuh"
 
 using namespace w4a8;
 
@@ -347,6 +348,107 @@ w4a8_status check_moe(int T, int E, int topk, const w4a8_wdesc* w1, const w4a8_w
     if (H % 64 != 0 || I % 64 != 0 || H > 8192 || I > 8192) return W4A8_ERR_UNSUPPORTED_SHAPE;
     if ((long long)T * topk > (1ll << 26)) return W4A8_ERR_UNSUPPORTED_SHAPE;
     return W4A8_OK;
+}
+
+// ------------------------------------------------------------------ W8A8 --
+
+// A W8A8 weight descriptor: bits 8, one group spanning K (per-channel scale).
+w4a8_status check_w8desc(const w4a8_wdesc* w) {
+    if (!w) return W4A8_ERR_INVALID_ARG;
+    if (w->bits != 8 || w->layout_version != W4A8_LAYOUT_VERSION || w->symmetric != 1 || w->group != w->K)
+        return W4A8_ERR_FORMAT_MISMATCH;
+    if (w->K <= 0 || w->N <= 0 || w->K % 128 != 0 || w->N % 16 != 0) return W4A8_ERR_FORMAT_MISMATCH;
+    return W4A8_OK;
+}
+
+// Launch plan of the W8A8 GEMM: (tile, k-block of 128) units over a
+// persistent grid, split-K when the tiles do not fill the SMs.
+struct W8Plan {
+    int bn, m_tiles, n_tiles, KB, grid, slots;
+    long long Q;
+    bool split;
+    size_t flags_off, ws_bytes;
+};
+
+W8Plan plan_w8(int M, int N, int K, int sms) {
+    W8Plan pl{};
+    pl.bn = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256;
+    pl.m_tiles = (M + pl.bn - 1) / pl.bn;
+    pl.n_tiles = (N + 127) / 128;
+    pl.KB = K / 128;
+    const long long tiles = (long long)pl.m_tiles * pl.n_tiles;
+    const long long U = tiles * pl.KB;
+    if (sms <= 0) sms = 1;
+    const long long waves = (tiles + sms - 1) / sms;
+    const double eff = (double)tiles / (double)(waves * sms);
+    pl.split = (eff < 0.85) && pl.KB > 1;
+    if (pl.split) {
+        pl.Q = (U + sms - 1) / sms;
+        pl.grid = (int)((U + pl.Q - 1) / pl.Q);
+        pl.slots = (int)((pl.KB + pl.Q - 1) / pl.Q) + 1;
+        pl.flags_off = align_up((size_t)tiles * pl.slots * pl.bn * 128 * sizeof(int32_t), 256);
+        pl.ws_bytes = pl.flags_off + (size_t)tiles * pl.slots * sizeof(unsigned long long);
+    } else {
+        pl.Q = (long long)pl.KB * waves;
+        pl.grid = (int)((tiles + waves - 1) / waves);
+        pl.slots = 0;
+        pl.ws_bytes = 0;
+    }
+    return pl;
+}
+
+// 2-D tensor map over an int8 [rows][K] matrix, box 128 k x box_rows rows,
+// 128-byte swizzle (the MMA's K-major operand layout).
+bool make_k128_tmap(CUtensorMap* map, const void* base, long long rows, int K, int box_rows) {
+    EncodeTiledFn enc = get_encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)K};
+    cuuint32_t box[2] = {128, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+w4a8_status w8_gemm_impl(const int8_t* qx, const float* s_x, const int8_t* q_w, const float* s_w,
+                         const w4a8_wdesc* w, int M, uint16_t* Y, int ldy, void* workspace, size_t ws_bytes,
+                         int32_t* dev_status, void* stream) {
+    w4a8_status st = check_w8desc(w);
+    if (st != W4A8_OK) return st;
+    if (M < 0 || !Y || ldy < w->N) return W4A8_ERR_INVALID_ARG;
+    if (M == 0) return W4A8_OK;
+    if (!qx || !s_x || !q_w || !s_w) return W4A8_ERR_INVALID_ARG;
+    if (!aligned16(qx) || !aligned16(q_w)) return W4A8_ERR_INVALID_ARG;
+    if (w->K > (1 << 17) || M > (1 << 24)) return W4A8_ERR_UNSUPPORTED_SHAPE;  // |acc| < 2^31
+    const W8Plan pl = plan_w8(M, w->N, w->K, sm_count_current());
+    if (pl.ws_bytes > 0 && (!workspace || ws_bytes < pl.ws_bytes)) return W4A8_ERR_WORKSPACE;
+    CUtensorMap tw, tx;
+    if (!make_k128_tmap(&tw, q_w, w->N, w->K, 128) || !make_k128_tmap(&tx, qx, M, w->K, pl.bn)) return W4A8_ERR_CUDA;
+    W8Params p{};
+    p.N = w->N;
+    p.K = w->K;
+    p.M = M;
+    p.n_tiles = pl.n_tiles;
+    p.m_tiles = pl.m_tiles;
+    p.KB = pl.KB;
+    p.units_per_cta = pl.Q;
+    p.s_w = s_w;
+    p.s_x = s_x;
+    p.Y = Y;
+    p.ldy = ldy;
+    p.vec16 = (aligned16(Y) && ldy % 8 == 0) ? 1 : 0;
+    p.partial = static_cast<int32_t*>(workspace);
+    p.slots = pl.slots;
+    if (pl.split) {
+        p.flags = reinterpret_cast<unsigned long long*>(static_cast<uint8_t*>(workspace) + pl.flags_off);
+        p.epoch = next_epoch();
+    }
+    p.status = dev_status;
+    p.wait_ns = kDefaultWaitNs;
+    return static_cast<w4a8_status>(
+        launch_w8a8(pl.bn, pl.split, tw, tx, p, pl.grid, static_cast<cudaStream_t>(stream)));
 }
 
 }  // namespace
@@ -709,6 +811,64 @@ w4a8_status w4a8_get_device_status(const int32_t* dev_status, void* stream) {
     int32_t v = 0;
     if (cudaMemcpy(&v, dev_status, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) return W4A8_ERR_CUDA;
     return static_cast<w4a8_status>(v);
+}
+
+w4a8_status w8a8_pack_weights(const float* W, int K, int N, int8_t* q_w, float* s_w, w4a8_wdesc* out,
+                              int32_t* dev_status, void* stream) {
+    if (!W || !q_w || !s_w) return W4A8_ERR_INVALID_ARG;
+    if (K <= 0 || N <= 0 || K % 128 != 0 || N % 16 != 0) return W4A8_ERR_INVALID_ARG;
+    if (!aligned16(q_w)) return W4A8_ERR_INVALID_ARG;
+    pack_w8_kernel<<<(unsigned)((N + 127) / 128), 128, 0, static_cast<cudaStream_t>(stream)>>>(W, K, N, q_w, s_w,
+                                                                                              dev_status);
+    w4a8_status st = last_cuda();
+    if (st == W4A8_OK && out) {
+        out->bits = 8;
+        out->symmetric = 1;
+        out->group = K;
+        out->K = K;
+        out->N = N;
+        out->layout_version = W4A8_LAYOUT_VERSION;
+    }
+    return st;
+}
+
+size_t w8a8_gemm_workspace_size(int M, const w4a8_wdesc* w) {
+    if (M <= 0 || check_w8desc(w) != W4A8_OK) return 0;
+    return plan_w8(M, w->N, w->K, sm_count_current()).ws_bytes;
+}
+
+w4a8_status w8a8_gemm(const int8_t* qx, const float* s_x, const int8_t* q_w, const float* s_w, const w4a8_wdesc* w,
+                      int M, uint16_t* Y, int ldy, void* workspace, size_t ws_bytes, int32_t* dev_status,
+                      void* stream) {
+    return w8_gemm_impl(qx, s_x, q_w, s_w, w, M, Y, ldy, workspace, ws_bytes, dev_status, stream);
+}
+
+size_t w8a8_linear_workspace_size(int M, const w4a8_wdesc* w) {
+    if (M <= 0 || check_w8desc(w) != W4A8_OK) return 0;
+    const size_t sx = align_up((size_t)M * w->K, 256);
+    const size_t g = align_up(sx + sizeof(float) * (size_t)M, 256);
+    return g + plan_w8(M, w->N, w->K, sm_count_current()).ws_bytes;
+}
+
+w4a8_status w8a8_linear(const uint16_t* X, int M, int ldx, const int8_t* q_w, const float* s_w, const w4a8_wdesc* w,
+                        uint16_t* Y, int ldy, void* workspace, size_t ws_bytes, int32_t* dev_status, void* stream) {
+    w4a8_status st = check_w8desc(w);
+    if (st != W4A8_OK) return st;
+    if (M < 0 || !Y || ldy < w->N) return W4A8_ERR_INVALID_ARG;
+    if (M == 0) return W4A8_OK;
+    if (!X || ldx < w->K) return W4A8_ERR_INVALID_ARG;
+    if (ldx % 8 != 0 || !aligned16(X)) return W4A8_ERR_UNSUPPORTED_SHAPE;
+    const size_t need = w8a8_linear_workspace_size(M, w);
+    if (!workspace || ws_bytes < need || !aligned16(workspace)) return W4A8_ERR_WORKSPACE;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    const size_t sxo = align_up((size_t)M * w->K, 256);
+    const size_t go = align_up(sxo + sizeof(float) * (size_t)M, 256);
+    int8_t* qx = reinterpret_cast<int8_t*>(ws);
+    float* sx = reinterpret_cast<float*>(ws + sxo);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    st = launch_quant(X, M, w->K, ldx, qx, sx, nullptr, 0, nullptr, 0, dev_status, s);
+    if (st != W4A8_OK) return st;
+    return w8_gemm_impl(qx, sx, q_w, s_w, w, M, Y, ldy, ws + go, ws_bytes - go, dev_status, stream);
 }
 
 w4a8_status w4a8_selftest_bounded_wait(int32_t* dev_status, uint64_t limit_ns, void* stream) {

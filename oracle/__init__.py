@@ -326,3 +326,43 @@ def moe_forward(X_bf16, logits, topk, experts_w1, experts_w2, group):
     return dict(idx=idx, p=p, offsets=offsets, perm=perm, inv=inv, qx=qx, sx=sx,
                 q_perm=q_perm, s_perm=s_perm, H=H_gu, h=h, qh=qh, sh=sh, Yd64=Yd64,
                 Yd=Yd, out=out, out64=out64, P1=P1, P2=P2, nonfinite=bad_l or bad_x)
+
+
+# --------------------------------------------------------------------------
+# W8A8: per-channel INT8 weights ("Inference Quantization ch.1" §2, §4, §8.2)
+# --------------------------------------------------------------------------
+
+def quant_w8(W: np.ndarray):
+    """Per-channel INT8 weight quantization of W fp32 [K,N]: every column n is
+    quantized like a token row (the W8A16 worked example of §2 quantizes a
+    weight vector with s = max|W| / 127, q = round(W / s)).  Returns
+    (q int8 [K,N], s_w fp32 [N], nonfinite flag)."""
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    K, N = W.shape
+    q = np.empty((K, N), dtype=np.int8)
+    s = np.empty(N, dtype=np.float32)
+    bad = False
+    for n in range(N):
+        qc, sc, b = quant_row_f32(np.ascontiguousarray(W[:, n]))
+        q[:, n] = qc
+        s[n] = sc
+        bad |= b
+    return q, s, bad
+
+
+def w8a8_exact(qx: np.ndarray, s_x: np.ndarray, qw: np.ndarray, s_w: np.ndarray):
+    """§4 ideal path, §8.3: Y = s_x[m] s_w[n] sum_k q_x[m,k] q_w[k,n] with the
+    integer sum exact (int64 matmul) and the scaling in binary64.  Returns
+    (Y fp64 [M,N], sum of |terms| fp64 [M,N] for the tolerance, acc int64)."""
+    acc = qx.astype(np.int64) @ qw.astype(np.int64)
+    absacc = np.abs(qx.astype(np.int64)) @ np.abs(qw.astype(np.int64))
+    sc = s_x.astype(np.float64)[:, None] * s_w.astype(np.float64)[None, :]
+    return sc * acc.astype(np.float64), np.abs(sc) * absacc.astype(np.float64), acc
+
+
+def w8a8_dequant_gemm(qx: np.ndarray, s_x: np.ndarray, qw: np.ndarray, s_w: np.ndarray) -> np.ndarray:
+    """The same product computed the other way round (dequantize both operands
+    in binary64, then multiply): the identity the factorised form must meet."""
+    Xd = s_x.astype(np.float64)[:, None] * qx.astype(np.float64)
+    Wd = qw.astype(np.float64) * s_w.astype(np.float64)[None, :]
+    return Xd @ Wd

@@ -457,3 +457,60 @@ def test_moe_forward_tiny_against_dense_dequant():
             yd = O.dequant_gemm(qh, sh, *w2[e], g)[0]
             acc += r["p"][t, j] * O.bf16_to_f32(O.f64_to_bf16(yd)).astype(np.float64)
         assert np.allclose(acc, r["out64"][t], rtol=1e-12, atol=1e-12)
+
+
+# ------------------------------------------------------- W8A8 per-channel --
+
+def test_w8_per_channel_worked_example_linear_s2(orc, golden):
+    """The §2 worked example quantizes a weight vector: as one output column
+    of W it must give the printed codes and scale."""
+    g = golden("lin_s2_worked_int8.txt")
+    W = np.array([[float(v)] for v in g["input"]], np.float32)  # [K=4, N=1]
+    q, s, bad = orc.quant_w8(W)
+    assert not bad
+    assert q[:, 0].tolist() == [int(v) for v in g["codes"]]
+    assert round(float(s[0]), 4) == float(g["scale_printed"][0])
+
+
+def test_w8_columns_are_independent_and_zero_column():
+    """Per-channel: scaling one column by a power of two scales its s_w and
+    leaves its codes and every other column unchanged; an all-zero column
+    gives s = 0 and codes 0 (the zero-scale reading)."""
+    import oracle as O
+    rng = np.random.default_rng(3)
+    W = (rng.standard_normal((256, 5)) * 0.02).astype(np.float32)
+    W[:, 2] = 0.0
+    q, s, _ = O.quant_w8(W)
+    W2 = W.copy()
+    W2[:, 1] *= 8.0
+    q2, s2, _ = O.quant_w8(W2)
+    assert np.array_equal(q, q2)
+    assert s2[1] == np.float32(8.0) * s[1]
+    assert np.array_equal(np.delete(s, 1), np.delete(s2, 1))
+    assert s[2] == 0.0 and not q[:, 2].any()
+    assert np.abs(q).max() <= 127 and (np.abs(q).max(axis=0)[[0, 1, 3, 4]] == 127).all()
+
+
+def test_w8a8_factorised_equals_dequantize_then_gemm():
+    """§4: s_x s_w (X_int8 W_int8) equals the product of the dequantized
+    operands (both in binary64; the integer sum is exact)."""
+    import oracle as O
+    rng = np.random.default_rng(4)
+    qx = rng.integers(-127, 128, size=(7, 384)).astype(np.int8)
+    qw = rng.integers(-127, 128, size=(384, 33)).astype(np.int8)
+    sx = rng.uniform(1e-3, 1e-1, size=7).astype(np.float32)
+    sw = rng.uniform(1e-4, 1e-2, size=33).astype(np.float32)
+    Y, A, _ = O.w8a8_exact(qx, sx, qw, sw)
+    Yd = O.w8a8_dequant_gemm(qx, sx, qw, sw)
+    assert np.all(np.abs(Y - Yd) <= 1e-12 * A)
+
+
+def test_w8a8_integer_sum_brute_force():
+    import oracle as O
+    rng = np.random.default_rng(5)
+    qx = rng.integers(-127, 128, size=(3, 20)).astype(np.int8)
+    qw = rng.integers(-127, 128, size=(20, 4)).astype(np.int8)
+    _, _, acc = O.w8a8_exact(qx, np.ones(3, np.float32), qw, np.ones(4, np.float32))
+    for m in range(3):
+        for n in range(4):
+            assert acc[m, n] == sum(int(qx[m, k]) * int(qw[k, n]) for k in range(20))
