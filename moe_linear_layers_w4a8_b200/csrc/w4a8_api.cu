@@ -4,6 +4,7 @@
 // (tile shape, persistent grid, split-K), TMA descriptor encoding, and the
 // launches.  Every call is asynchronous on the caller's stream and never
 // allocates; scratch lives in the caller's workspace.
+#include <algorithm>
 #include <atomic>
 #include <chrono>
 #include <random>
@@ -647,6 +648,9 @@ w4a8_status moe_impl(const uint16_t* X, const float* logits, int T, int E, int t
     uint16_t* yd = reinterpret_cast<uint16_t*>(ws + L.yd);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int R = T * topk;
+    // Token tile width from the mean rows per expert (measured on the T=64,
+    // E=256 top-8 layer: BN = 16 with several m-tiles for the hot experts is
+    // faster than one BN = 64 tile per expert, 0.45 vs 0.62 ms for gate_up).
     const int bn = pick_bn(((long long)R + E - 1) / E);
     auto mark = [&](int i) -> bool {
         if (!stage_events || !stage_events[i]) return true;
