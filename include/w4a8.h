@@ -390,6 +390,45 @@ W4A8_API w4a8_status w4a8_moe_debug_partials(
     void* workspace, size_t ws_bytes, int32_t* dev_status, void* stream,
     const int32_t* pair_slot, int32_t* P1, int32_t* P2);
 
+/* ------------------------------------------- expert-parallel building blocks -- */
+
+/*
+ * The three pieces of w4a8_moe_grouped_gemm that an expert-parallel layer
+ * ("Kimi 2.7 MoE W4A8 deployment in practice" §5.4: experts spread over
+ * GPUs, tokens exchanged all-to-all) runs on different ranks: routing on the
+ * rank that holds the tokens, the expert GEMMs on the rank that holds the
+ * experts, the weighted combine back on the tokens' rank.  Composed in that
+ * order with the rows exchanged in between, they compute exactly what
+ * w4a8_moe_grouped_gemm computes (the same kernels, the same rounding).
+ */
+
+/* w4a8_moe_route — step 1 alone: topk_idx_out int32 [T][topk], topk_w_out
+ * fp32 [T][topk] from logits fp32 [T][E] (device). */
+W4A8_API w4a8_status w4a8_moe_route(const float* logits, int T, int E, int topk, int32_t* topk_idx_out,
+                                    float* topk_w_out, int32_t* dev_status, void* stream);
+
+/* Workspace bytes w4a8_moe_experts needs for R rows. */
+W4A8_API size_t w4a8_moe_experts_workspace_size(int R, int E, const w4a8_wdesc* w1, const w4a8_wdesc* w2);
+
+/* w4a8_moe_experts — steps 2-6 for rows whose expert is already chosen: row
+ * r of X bf16 [R][H] goes through expert expert_ids[r] (device int32 [R], in
+ * [0, E): the experts stacked in w1_* / w2_* as for w4a8_moe_grouped_gemm);
+ * y_out bf16 [R][H] receives each row's expert output, unweighted (bf16, as
+ * the layer stores expert outputs before its combine).  An id outside [0, E)
+ * is reported as W4A8_ERR_INVALID_ARG through dev_status.  Limits and errors
+ * as w4a8_moe_grouped_gemm. */
+W4A8_API w4a8_status w4a8_moe_experts(const uint16_t* X, const int32_t* expert_ids, int R, int E,
+                                      const uint8_t* w1_packed, const float* w1_s, const uint8_t* w1_z,
+                                      const w4a8_wdesc* w1, const uint8_t* w2_packed, const float* w2_s,
+                                      const uint8_t* w2_z, const w4a8_wdesc* w2, uint16_t* y_out, void* workspace,
+                                      size_t ws_bytes, int32_t* dev_status, void* stream);
+
+/* w4a8_moe_combine — step 7 alone: out[t] = sum_j topk_w[t,j] * y_rows[t*topk
+ * + j] in fp32, slot order, one bf16 rounding (y_rows bf16 [T*topk][H] in
+ * (token, slot) order; H % 8 == 0; y_rows and out 16-byte aligned). */
+W4A8_API w4a8_status w4a8_moe_combine(const uint16_t* y_rows, const float* topk_w, int T, int topk, int H,
+                                      uint16_t* out, void* stream);
+
 /* --------------------------------------------------------------- status -- */
 
 /* Synchronizes `stream`, then reads the device status word (0 = W4A8_OK).

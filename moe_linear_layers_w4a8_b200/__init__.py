@@ -23,7 +23,7 @@ __all__ = [
     "w4a8_gemm_workspace_size", "w4a8_moe_workspace_size", "w4a8_get_device_status",
     "w4a8_status_string", "w4a8_selftest_bounded_wait", "w4a8_linear", "w4a8_linear_workspace_size", "LAYOUT_VERSION",
     "STATUS", "PackedW8", "w8a8_pack_weights", "w8a8_gemm", "w8a8_gemm_workspace_size", "w8a8_linear",
-    "w8a8_linear_workspace_size",
+    "w8a8_linear_workspace_size", "w4a8_moe_route", "w4a8_moe_experts", "w4a8_moe_combine",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -124,6 +124,15 @@ def load_library():
         L.w4a8_moe_grouped_gemm_profiled.argtypes = L.w4a8_moe_grouped_gemm.argtypes + [P]
         L.w4a8_moe_debug_partials.restype = st
         L.w4a8_moe_debug_partials.argtypes = L.w4a8_moe_grouped_gemm.argtypes + [P, P, P]
+        L.w4a8_moe_route.restype = st
+        L.w4a8_moe_route.argtypes = [P, I, I, I, P, P, P, P]
+        L.w4a8_moe_experts_workspace_size.restype = S
+        L.w4a8_moe_experts_workspace_size.argtypes = [I, I, ctypes.POINTER(WDesc), ctypes.POINTER(WDesc)]
+        L.w4a8_moe_experts.restype = st
+        L.w4a8_moe_experts.argtypes = [P, P, I, I, P, P, P, ctypes.POINTER(WDesc), P, P, P, ctypes.POINTER(WDesc),
+                                       P, P, S, P, P]
+        L.w4a8_moe_combine.restype = st
+        L.w4a8_moe_combine.argtypes = [P, P, I, I, I, P, P]
         L.w8a8_pack_weights.restype = st
         L.w8a8_pack_weights.argtypes = [P, I, I, P, P, ctypes.POINTER(WDesc), P, P]
         L.w8a8_gemm_workspace_size.restype = S
@@ -474,4 +483,59 @@ def w8a8_linear(X: torch.Tensor, w: PackedW8, out=None, workspace=None, status=N
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(L.w8a8_linear(_p(X), M, X.stride(0), _p(w.q_w), _p(w.s_w), ctypes.byref(w.desc), _p(out), out.stride(0),
                          _p(workspace), ws_bytes, _p(status), _stream(X.device)), "w8a8_linear")
+    return out
+
+
+# ------------------------------------------- expert-parallel building blocks --
+
+def w4a8_moe_route(logits: torch.Tensor, topk: int, status: Optional[torch.Tensor] = None):
+    """(topk_idx int32 [T, k], topk_w fp32 [T, k]) of logits fp32 [T, E]."""
+    L = load_library()
+    _need_cuda(logits)
+    logits = logits.contiguous()
+    T, E = logits.shape
+    idx = torch.empty(T, topk, dtype=torch.int32, device=logits.device)
+    w = torch.empty(T, topk, dtype=torch.float32, device=logits.device)
+    _check(L.w4a8_moe_route(_p(logits), T, E, int(topk), _p(idx), _p(w), _p(status), _stream(logits.device)),
+           "w4a8_moe_route")
+    return idx, w
+
+
+def w4a8_moe_experts(X: torch.Tensor, expert_ids: torch.Tensor, w1: PackedWeight, w2: PackedWeight,
+                     workspace: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None,
+                     out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """y bf16 [R, H]: row r of X bf16 [R, H] through expert expert_ids[r] (unweighted)."""
+    L = load_library()
+    _need_cuda(X, expert_ids)
+    X = X.contiguous()
+    ids = expert_ids.to(torch.int32).contiguous()
+    R, H = X.shape
+    E = w1.experts
+    if out is None:
+        out = torch.empty(R, H, dtype=torch.bfloat16, device=X.device)
+    if R == 0:
+        return out
+    need = int(L.w4a8_moe_experts_workspace_size(R, E, ctypes.byref(w1.desc), ctypes.byref(w2.desc)))
+    if need == 0:
+        raise W4A8Error(2, "w4a8_moe_experts_workspace_size: shape not supported")
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=X.device)
+    _check(L.w4a8_moe_experts(_p(X), _p(ids), R, E, _p(w1.packed), _p(w1.s_w), _p(w1.z), ctypes.byref(w1.desc),
+                              _p(w2.packed), _p(w2.s_w), _p(w2.z), ctypes.byref(w2.desc), _p(out), _p(workspace),
+                              workspace.numel() * workspace.element_size(), _p(status), _stream(X.device)),
+           "w4a8_moe_experts")
+    return out
+
+
+def w4a8_moe_combine(y_rows: torch.Tensor, topk_w: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """out bf16 [T, H] = sum_j topk_w[t, j] * y_rows[t * k + j] (fp32, slot order)."""
+    L = load_library()
+    _need_cuda(y_rows, topk_w)
+    T, k = topk_w.shape
+    H = y_rows.shape[1]
+    y_rows = y_rows.contiguous()
+    topk_w = topk_w.contiguous()
+    if out is None:
+        out = torch.empty(T, H, dtype=torch.bfloat16, device=y_rows.device)
+    _check(L.w4a8_moe_combine(_p(y_rows), _p(topk_w), T, k, H, _p(out), _stream(y_rows.device)), "w4a8_moe_combine")
     return out

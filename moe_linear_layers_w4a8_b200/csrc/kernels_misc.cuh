@@ -636,7 +636,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
     for (int j = 0; j < topk; ++j) {
-        const int r = __ldg(inv + (size_t)t * topk + j);
+        // inv == null: the rows are already in (token, slot) order
+        const int r = inv ? __ldg(inv + (size_t)t * topk + j) : t * topk + j;
         const float w = __ldg(p + (size_t)t * topk + j);
         const uint4 v = __ldg(reinterpret_cast<const uint4*>(Yd + (size_t)r * H) + c);
         const uint32_t ws[4] = {v.x, v.y, v.z, v.w};
@@ -688,6 +689,26 @@ __global__ void __launch_bounds__(128) pack_w8_kernel(const float* __restrict__ 
     }
     s_w[n] = s;
     if (bad) report_status(status, kStatusNonfinite);
+}
+
+// Pre-routed expert rows (expert parallelism: the routing ran on another
+// rank): copies the expert id of every row into the routing output with
+// weight 1, so the layer's dispatch / expert GEMMs / combine run unchanged
+// and the combine returns each row's expert output as is.  An id outside
+// [0, E) is reported (W4A8_ERR_INVALID_ARG) and replaced by 0, so every later
+// index stays in bounds.
+__global__ void __launch_bounds__(256) preroute_kernel(const int32_t* __restrict__ ids, int R, int E,
+                                                       int32_t* __restrict__ idx, float* __restrict__ w,
+                                                       int32_t* status) {
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= R) return;
+    int e = __ldg(ids + i);
+    if (e < 0 || e >= E) {
+        report_status(status, 1);
+        e = 0;
+    }
+    idx[i] = e;
+    w[i] = 1.0f;
 }
 
 // Test hook: one warp waits on a barrier nobody arrives on.

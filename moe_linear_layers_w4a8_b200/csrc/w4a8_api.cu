@@ -618,11 +618,12 @@ w4a8_status moe_impl(const uint16_t* X, const float* logits, int T, int E, int t
                      const float* w2_s, const uint8_t* w2_z, const w4a8_wdesc* w2, uint16_t* out,
                      int32_t* topk_idx_out, float* topk_w_out, int32_t* expert_offsets_out, void* workspace,
                      size_t ws_bytes, int32_t* dev_status, void* stream, void* const* stage_events,
-                     const int32_t* dbg_map, int32_t* P1, int32_t* P2) {
+                     const int32_t* dbg_map, int32_t* P1, int32_t* P2, const int32_t* pre_ids = nullptr) {
     w4a8_status st = check_moe(T, E, topk, w1, w2);
     if (st != W4A8_OK) return st;
     if (T == 0) return W4A8_OK;
-    if (!X || !logits || !w1_packed || !w1_s || !w2_packed || !w2_s || !out || !topk_idx_out || !topk_w_out ||
+    if (pre_ids && topk != 1) return W4A8_ERR_INVALID_ARG;
+    if (!X || !(logits || pre_ids) || !w1_packed || !w1_s || !w2_packed || !w2_s || !out || !topk_idx_out || !topk_w_out ||
         !expert_offsets_out)
         return W4A8_ERR_INVALID_ARG;
     const bool sym = w1->symmetric != 0;
@@ -658,9 +659,13 @@ w4a8_status moe_impl(const uint16_t* X, const float* logits, int T, int E, int t
                cudaSuccess;
     };
 
-    // 1. routing
+    // 1. routing (or the given expert of each row)
     if (!mark(0)) return W4A8_ERR_CUDA;
-    {
+    if (pre_ids) {
+        preroute_kernel<<<(unsigned)((T + 255) / 256), 256, 0, s>>>(pre_ids, T, E, topk_idx_out, topk_w_out,
+                                                                    dev_status);
+        if ((st = last_cuda()) != W4A8_OK) return st;
+    } else {
         const int epl = (E + 31) / 32;
         const unsigned blocks = (unsigned)(((long long)T * 32 + 255) / 256);
         switch (epl) {
@@ -806,6 +811,60 @@ w4a8_status w4a8_moe_grouped_gemm(const uint16_t* X, const float* logits, int T,
     return w4a8_moe_grouped_gemm_profiled(X, logits, T, E, topk, w1_packed, w1_s, w1_z, w1, w2_packed, w2_s, w2_z,
                                           w2, out, topk_idx_out, topk_w_out, expert_offsets_out, workspace,
                                           ws_bytes, dev_status, stream, nullptr);
+}
+
+w4a8_status w4a8_moe_route(const float* logits, int T, int E, int topk, int32_t* topk_idx_out, float* topk_w_out,
+                           int32_t* dev_status, void* stream) {
+    if (T < 0 || E <= 0 || topk <= 0 || topk > E || E > kMaxExperts || topk > 16) return W4A8_ERR_INVALID_ARG;
+    if (T == 0) return W4A8_OK;
+    if (!logits || !topk_idx_out || !topk_w_out) return W4A8_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int epl = (E + 31) / 32;
+    const unsigned blocks = (unsigned)(((long long)T * 32 + 255) / 256);
+    switch (epl) {
+#define W4A8_ROUTE(n) case n: route_topk_kernel<n><<<blocks, 256, 0, s>>>(logits, T, E, topk, topk_idx_out, topk_w_out, dev_status); break;
+        W4A8_ROUTE(1) W4A8_ROUTE(2) W4A8_ROUTE(3) W4A8_ROUTE(4) W4A8_ROUTE(5) W4A8_ROUTE(6) W4A8_ROUTE(7)
+        W4A8_ROUTE(8) W4A8_ROUTE(9) W4A8_ROUTE(10) W4A8_ROUTE(11) W4A8_ROUTE(12) W4A8_ROUTE(13)
+        W4A8_ROUTE(14) W4A8_ROUTE(15) W4A8_ROUTE(16)
+#undef W4A8_ROUTE
+        default: return W4A8_ERR_UNSUPPORTED_SHAPE;
+    }
+    return last_cuda();
+}
+
+size_t w4a8_moe_experts_workspace_size(int R, int E, const w4a8_wdesc* w1, const w4a8_wdesc* w2) {
+    if (check_moe(R, E, 1, w1, w2) != W4A8_OK) return 0;
+    return moe_layout(R, E, 1, w1->K, w1->N / 2).total + align_up(sizeof(int32_t) * (size_t)(2 * R + E + 1), 256);
+}
+
+w4a8_status w4a8_moe_experts(const uint16_t* X, const int32_t* expert_ids, int R, int E, const uint8_t* w1_packed,
+                             const float* w1_s, const uint8_t* w1_z, const w4a8_wdesc* w1, const uint8_t* w2_packed,
+                             const float* w2_s, const uint8_t* w2_z, const w4a8_wdesc* w2, uint16_t* y_out,
+                             void* workspace, size_t ws_bytes, int32_t* dev_status, void* stream) {
+    w4a8_status st = check_moe(R, E, 1, w1, w2);
+    if (st != W4A8_OK) return st;
+    if (R == 0) return W4A8_OK;
+    if (!expert_ids) return W4A8_ERR_INVALID_ARG;
+    const size_t base = moe_layout(R, E, 1, w1->K, w1->N / 2).total;
+    if (!workspace || ws_bytes < w4a8_moe_experts_workspace_size(R, E, w1, w2)) return W4A8_ERR_WORKSPACE;
+    // the routing outputs of the layer (expert id, weight 1, offsets) live past the layer's own workspace
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    int32_t* idx = reinterpret_cast<int32_t*>(ws + base);
+    float* wts = reinterpret_cast<float*>(idx + R);
+    int32_t* offs = reinterpret_cast<int32_t*>(wts + R);
+    return moe_impl(X, nullptr, R, E, 1, w1_packed, w1_s, w1_z, w1, w2_packed, w2_s, w2_z, w2, y_out, idx, wts, offs,
+                    workspace, base, dev_status, stream, nullptr, nullptr, nullptr, nullptr, expert_ids);
+}
+
+w4a8_status w4a8_moe_combine(const uint16_t* y_rows, const float* topk_w, int T, int topk, int H, uint16_t* out,
+                             void* stream) {
+    if (T < 0 || topk <= 0 || H <= 0 || H % 8 != 0) return W4A8_ERR_INVALID_ARG;
+    if (T == 0) return W4A8_OK;
+    if (!y_rows || !topk_w || !out || !aligned16(y_rows) || !aligned16(out)) return W4A8_ERR_INVALID_ARG;
+    const long long n = (long long)T * (H / 8);
+    combine_kernel<<<(unsigned)((n + 255) / 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        y_rows, topk_w, nullptr, T, topk, H, out);
+    return last_cuda();
 }
 
 w4a8_status w4a8_get_device_status(const int32_t* dev_status, void* stream) {

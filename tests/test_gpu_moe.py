@@ -293,3 +293,35 @@ def test_moe_asym_prefill_config(m):
     tokens = sample_tokens(T, 10, 2, extra=[0, 4095, T - 1])
     res = run_layer(m, layer, inp, topk, tokens=tokens)
     check_layer(m, layer, inp, topk, res, tokens=tokens)
+
+
+@pytest.mark.parametrize("T,H,E,topk,I,g,sym,zipf", [(200, 256, 16, 4, 128, 128, True, 1.1),
+                                                      (64, 512, 8, 2, 192, 64, False, None)])
+def test_moe_building_blocks_equal_layer(m, T, H, E, topk, I, g, sym, zipf):
+    """Routing, pre-routed experts and combine run as separate calls (the
+    expert-parallel layer with one rank) give w4a8_moe_grouped_gemm's result
+    bit for bit."""
+    from moe_linear_layers_w4a8_b200.ep import ExpertParallelMoE
+    layer = Layer(m, seed=T + E, E=E, H=H, I=I, group=g, sym=sym, w_outlier_p=0.001)
+    inp = gen_moe_activations(T, H, E, seed=T * 5 + E, zipf=zipf)
+    X, L = inp.X.cuda(), inp.logits.cuda()
+    res = run_layer(m, layer, inp, topk)
+    ep = ExpertParallelMoE(E, layer.w1, layer.w2)
+    out, idx, w = ep.forward(X, L, topk)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, res["topk_idx"])
+    assert torch.equal(w, res["topk_w"])
+    assert np.array_equal(bits(out), bits(res["out"]))
+
+
+def test_moe_experts_rejects_out_of_range_ids(m):
+    T, H, E, I = 16, 128, 4, 64
+    layer = Layer(m, seed=3, E=E, H=H, I=I, group=64, sym=True, w_outlier_p=0.0)
+    X = gen_moe_activations(T, H, E, seed=3).X.cuda()
+    ids = torch.full((T,), 1, dtype=torch.int32, device="cuda")
+    ids[5] = E + 3
+    st = m.new_status("cuda")
+    m.w4a8_moe_experts(X, ids, layer.w1, layer.w2, status=st)
+    assert m.w4a8_get_device_status(st) == 1
+    x = torch.ones(4, device="cuda")
+    assert float(x.sum()) == 4.0  # the context is still usable
