@@ -55,7 +55,8 @@ METRIC = "W4A8 GEMM TOPS (prefill) & weight GB/s (decode) vs B200 roofline; MoE 
 L2_BYTES = 126 * 1024 * 1024
 
 DEFAULT_STEPS = {"decode": 20000, "prefill": 1500, "moe_sym": 2000, "moe_asym_decode": 400,
-                 "moe_asym_prefill": 200, "w8a8_decode": 20000, "w8a8_prefill": 1500}
+                 "moe_asym_prefill": 200, "w8a8_decode": 20000, "w8a8_prefill": 1500,
+                 "w4a16_decode": 20000, "w4a16_prefill": 1500}
 
 
 # ---------------------------------------------------------------- peaks ---
@@ -140,8 +141,9 @@ class LinearWorkload:
     def __init__(self, name, M, K=4096, N=14336, group=128, device="cuda"):
         self.name, self.M, self.K, self.N, self.group = name, M, K, N, group
         self.dev = device
-        self.decode = name in ("decode", "w8a8_decode")
+        self.decode = name.endswith("decode")
         self.w8 = name.startswith("w8a8")  # per-channel INT8 weights (the W8A8 variant)
+        self.w16 = name.startswith("w4a16")  # bf16 activations, weights dequantized in the GEMM
 
     def setup(self):
         import torch
@@ -174,14 +176,19 @@ class LinearWorkload:
             ws = m.w8a8_gemm_workspace_size(M, pw)
             lws = m.w8a8_linear_workspace_size(M, pw)
             self._linear, self._gemm = m.w8a8_linear, m.w8a8_gemm
+        elif self.w16:
+            ws = lws = m.w4a16_gemm_workspace_size(M, pw)
+            self._linear = m.w4a16_gemm
+            self._gemm = lambda q, s, w, out, workspace: m.w4a16_gemm(self.X, w, out=out, workspace=workspace)
         else:
             ws = m.w4a8_gemm_workspace_size(M, pw)
             lws = m.w4a8_linear_workspace_size(M, pw)
             self._linear, self._gemm = m.w4a8_linear, m.w4a8_gemm
         self.ws = torch.empty(max(ws, 16), dtype=torch.uint8, device=self.dev)
-        self.lws = torch.empty(lws, dtype=torch.uint8, device=self.dev)
+        self.lws = torch.empty(max(lws, 16), dtype=torch.uint8, device=self.dev)
         self.splitk = ws > 0
-        self.launches_per_step = 2  # quantization + GEMM (split-K is summed inside the GEMM)
+        # quantization + GEMM (split-K is summed inside the GEMM); W4A16 has no quantization
+        self.launches_per_step = 1 if self.w16 else 2
 
     def step(self, i, ev=None):
         # the public one-call layer: the GEMM's weight streaming overlaps the quantization
@@ -190,14 +197,15 @@ class LinearWorkload:
     @property
     def kernel_timing_note(self):
         return (f"CUDA events around a graph of {self._chain} back-to-back "
-                f"{'w8a8_gemm' if self.w8 else 'w4a8_gemm'} launches "
-                f"(packed weights rotated, activations quantized once), mean per launch")
+                f"{'w8a8_gemm' if self.w8 else 'w4a16_gemm' if self.w16 else 'w4a8_gemm'} launches "
+                f"(packed weights rotated{'' if self.w16 else ', activations quantized once'}), mean per launch")
 
     def kernel_time(self, torch):
         """Per-launch duration of the GEMM: events around a chain of
         back-to-back launches in a CUDA graph (separate, untimed replays)."""
         m = self.m
-        m.w4a8_quant_act(self.X, q_out=self.q, s_out=self.s)
+        if not self.w16:
+            m.w4a8_quant_act(self.X, q_out=self.q, s_out=self.s)
         n = self._chain = 64 if self.decode else 8
 
         def chain(i, ev):
@@ -226,20 +234,28 @@ class LinearWorkload:
     def units(self):
         if self.decode:
             return self.w_bytes / 1e9, "GB/s", "weight+scale bytes streamed per second"
+        if self.w16:
+            return 2.0 * self.M * self.N * self.K / 1e12, "TFLOPS", "2*M*N*K bf16 flops per second"
         return 2.0 * self.M * self.N * self.K / 1e12, "TOPS", "2*M*N*K int8 ops per second"
 
     def kernel_roofline(self, peaks):
         M, K, N, g = self.M, self.K, self.N, self.group
         if self.decode:
-            alg = self.w_bytes + M * K + 4 * M + 2 * M * N
+            # weights + scales, activations (int8 + s_x, or bf16), bf16 output
+            alg = self.w_bytes + (2 * M * K if self.w16 else M * K + 4 * M) + 2 * M * N
             return dict(bound="hbm", per_launch=alg, unit="GB/s", scale=1e9, peak=peaks["hbm"],
                         peak_note=f"hbm_gbs ({peaks['source']})")
         ops = 2.0 * M * N * K
+        if self.w16:
+            return dict(bound="tensor", per_launch=ops, unit="TFLOP/s", scale=1e12, peak=peaks["bf16_sus"],
+                        peak_note=f"bf16_tflops_sustained ({peaks['source']})")
         return dict(bound="tensor", per_launch=ops, unit="TOPS", scale=1e12, peak=2.0 * peaks["bf16_sus"],
                     peak_note=f"2 x bf16_tflops_sustained ({peaks['source']}; int8/bf16 nominal ratio 2)")
 
     def config(self):
-        wfmt = "per-channel int8 weights (W8A8)" if self.w8 else f"symmetric int4 g={self.group}"
+        wfmt = ("per-channel int8 weights (W8A8)" if self.w8 else
+                f"symmetric int4 g={self.group}, bf16 activations (W4A16)" if self.w16 else
+                f"symmetric int4 g={self.group}")
         base = {"workload": f"{self.name} linear M={self.M} K={self.K} N={self.N} {wfmt}",
                 "M": self.M, "K": self.K, "N": self.N, "group": self.K if self.w8 else self.group}
         if not hasattr(self, "copies"):
@@ -274,6 +290,9 @@ class LinearWorkload:
         if self.w8:
             qw, sw, _ = O.quant_w8(W[:, cols].copy())  # offline step, untimed
             self._orc = (O, qw, sw, Xb)
+        elif self.w16:
+            codes, s, _, _ = O.quant_weights(W[:, cols].copy(), self.group, True)  # offline step, untimed
+            self._orc = (O, codes, s, Xb)
         else:
             codes, s, _, _ = O.quant_weights(W[:, cols].copy(), self.group, True)  # offline step, untimed
             self._orc = (O, codes, s, Xb)
@@ -288,6 +307,8 @@ class LinearWorkload:
         if self.w8:
             qx, sx, _, _ = O.quant_act(Xb)
             O.w8a8_exact(qx, sx, codes, s)
+        elif self.w16:
+            O.w4a16_gemm(Xb, O.w4a16_dequant(codes, s, None, self.group))
         else:
             O.linear(Xb, codes, s, None, self.group)
 
@@ -427,7 +448,7 @@ class MoEWorkload:
 
 
 def make_workload(name, M):
-    if name in ("decode", "prefill", "w8a8_decode", "w8a8_prefill"):
+    if name in ("decode", "prefill", "w8a8_decode", "w8a8_prefill", "w4a16_decode", "w4a16_prefill"):
         return LinearWorkload(name, M if M else (32 if name.endswith("decode") else 8192))
     return MoEWorkload(name)
 
@@ -597,7 +618,8 @@ def measure(args, wl, K, W, peaks, world, rank, local, cpu_budget_s):
     return out
 
 
-SECONDARY = ["prefill", "moe_sym", "moe_asym_decode", "moe_asym_prefill", "w8a8_decode", "w8a8_prefill"]
+SECONDARY = ["prefill", "moe_sym", "moe_asym_decode", "moe_asym_prefill", "w8a8_decode", "w8a8_prefill",
+             "w4a16_decode", "w4a16_prefill"]
 
 
 def run_ours(args, world, rank, local):
@@ -778,7 +800,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="decode",
                     choices=["decode", "prefill", "moe_sym", "moe_asym_decode", "moe_asym_prefill", "w8a8_decode",
-                             "w8a8_prefill"])
+                             "w8a8_prefill", "w4a16_decode", "w4a16_prefill"])
     ap.add_argument("--m", type=int, default=None, help="rows of the linear workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--main-only", action="store_true",

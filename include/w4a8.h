@@ -305,6 +305,43 @@ W4A8_API w4a8_status w8a8_linear(const uint16_t* X, int M, int ldx, const int8_t
                                  const w4a8_wdesc* w, uint16_t* Y, int ldy, void* workspace, size_t ws_bytes,
                                  int32_t* dev_status, void* stream);
 
+/* ------------------------------------------------------------ W4A16 ---- */
+
+/*
+ * The weight-only W4A16 variant ("Inference Quantization ch.1" §2 and §3.2:
+ * the activations stay bf16, the low-bit weights are dequantized inside the
+ * GEMM kernel and never written back as a full-precision tensor):
+ *   w_hat[k,n] = bf16( fp32( s_w[g,n] * (q[k,n] - z[g,n]) ) ),  g = k / group
+ *               (z = 0 for symmetric weights; one fp32 product, one bf16
+ *               rounding: the bf16 operand of the tensor-core MMA)
+ *   Y[m,n]     = bf16( sum_k X[m,k] * w_hat[k,n] )   fp32 accumulation
+ * Reads the W4A8 packed weights as they are (w4a8_pack_weights' packed, s_w,
+ * z and descriptor), so one packed copy serves both paths.
+ * The dequantization is exact for s_w >= 2^-110 (every scale of a weight
+ * group whose largest magnitude exceeds about 1e-32).
+ */
+
+/* Workspace bytes w4a16_gemm needs for M rows (split-K fp32 partial tiles and
+ * their flags; 0 when none). */
+W4A8_API size_t w4a16_gemm_workspace_size(int M, const w4a8_wdesc* w);
+
+/* w4a16_gemm — Y = X · dequant(packed W).
+ * X        device bf16 [M][ldx] row-major, 16-byte aligned, ldx % 8 == 0,
+ *          ldx >= K (read by TMA).
+ * packed, s_w, z, w: as produced by w4a8_pack_weights (z NULL iff
+ *          symmetric); packed, s_w and z 16-byte aligned.
+ * Y        device bf16 [M][ldy], ldy >= N.
+ * workspace / ws_bytes: at least w4a16_gemm_workspace_size(M, w) bytes of
+ *          device memory when that is > 0 (caller-owned, reused freely
+ *          between calls on one stream).  Split-K partial tiles are summed in
+ *          a fixed order, so results are deterministic.
+ * Errors: INVALID_ARG (null pointers, alignment, ldx/ldy), FORMAT_MISMATCH
+ *         (descriptor, z presence), UNSUPPORTED_SHAPE (K or M > 2^24),
+ *         WORKSPACE, CUDA; TIMEOUT via dev_status. */
+W4A8_API w4a8_status w4a16_gemm(const uint16_t* X, int M, int ldx, const uint8_t* packed, const float* s_w,
+                                const uint8_t* z, const w4a8_wdesc* w, uint16_t* Y, int ldy, void* workspace,
+                                size_t ws_bytes, int32_t* dev_status, void* stream);
+
 /*
  * w4a8_moe_grouped_gemm — one MoE expert layer, following "Kimi 2.7 MoE,
  * 4-bit storage to INT8" §4.1-4.4:

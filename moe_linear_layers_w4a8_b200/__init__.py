@@ -24,6 +24,7 @@ __all__ = [
     "w4a8_status_string", "w4a8_selftest_bounded_wait", "w4a8_linear", "w4a8_linear_workspace_size", "LAYOUT_VERSION",
     "STATUS", "PackedW8", "w8a8_pack_weights", "w8a8_gemm", "w8a8_gemm_workspace_size", "w8a8_linear",
     "w8a8_linear_workspace_size", "w4a8_moe_route", "w4a8_moe_experts", "w4a8_moe_combine",
+    "w4a16_gemm", "w4a16_gemm_workspace_size",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -143,6 +144,10 @@ def load_library():
         L.w8a8_linear_workspace_size.argtypes = [I, ctypes.POINTER(WDesc)]
         L.w8a8_linear.restype = st
         L.w8a8_linear.argtypes = [P, I, I, P, P, ctypes.POINTER(WDesc), P, I, P, S, P, P]
+        L.w4a16_gemm_workspace_size.restype = S
+        L.w4a16_gemm_workspace_size.argtypes = [I, ctypes.POINTER(WDesc)]
+        L.w4a16_gemm.restype = st
+        L.w4a16_gemm.argtypes = [P, I, I, P, P, P, ctypes.POINTER(WDesc), P, I, P, S, P, P]
         L.w4a8_get_device_status.restype = st
         L.w4a8_get_device_status.argtypes = [P, P]
         L.w4a8_selftest_bounded_wait.restype = st
@@ -483,6 +488,34 @@ def w8a8_linear(X: torch.Tensor, w: PackedW8, out=None, workspace=None, status=N
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(L.w8a8_linear(_p(X), M, X.stride(0), _p(w.q_w), _p(w.s_w), ctypes.byref(w.desc), _p(out), out.stride(0),
                          _p(workspace), ws_bytes, _p(status), _stream(X.device)), "w8a8_linear")
+    return out
+
+
+# ------------------------------------------------------------------ W4A16 --
+
+def w4a16_gemm_workspace_size(M: int, w: PackedWeight) -> int:
+    return int(load_library().w4a16_gemm_workspace_size(int(M), ctypes.byref(w.desc)))
+
+
+def w4a16_gemm(X: torch.Tensor, w: PackedWeight, out=None, workspace=None, status=None) -> torch.Tensor:
+    """Y bf16 [M, N] = X bf16 [M, K] times the W4A8-packed weight dequantized
+    to bf16 inside the kernel (the weight-only W4A16 path)."""
+    L = load_library()
+    _need_cuda(X)
+    if X.dtype != torch.bfloat16 or X.dim() != 2 or X.stride(1) != 1:
+        raise W4A8Error(1, "X must be bf16 [M, K] with unit column stride")
+    if w.experts:
+        raise W4A8Error(1, "w4a16_gemm takes one weight matrix, not stacked experts")
+    M = X.shape[0]
+    if out is None:
+        out = torch.empty(M, w.N, dtype=torch.bfloat16, device=X.device)
+    need = w4a16_gemm_workspace_size(M, w)
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=X.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    code = L.w4a16_gemm(_p(X), M, X.stride(0), _p(w.packed), _p(w.s_w), _p(w.z), ctypes.byref(w.desc), _p(out),
+                        out.stride(0), _p(workspace), ws_bytes, _p(status), _stream(X.device))
+    _check(code, "w4a16_gemm")
     return out
 
 

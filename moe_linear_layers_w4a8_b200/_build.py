@@ -12,7 +12,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libw4a8.so")
 SOURCES = [os.path.join(CSRC, f) for f in
            ("w4a8_api.cu", "gemm_plain.cu", "gemm_splitk.cu", "gemm_gateup.cu", "gemm_down.cu",
-            "gemm_w8a8.cu")]
+            "gemm_w8a8.cu", "gemm_w4a16.cu")]
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")] + [
     os.path.join(INCLUDE, "w4a8.h")]
 BUILD_DIR = os.path.join(PKG, "_build")

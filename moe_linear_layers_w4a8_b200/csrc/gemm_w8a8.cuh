@@ -134,10 +134,10 @@ __global__ void __launch_bounds__(kW8Threads, 1)
             long long issued = 0;
             bool ok = true;
             bool waited = false;
-            for (long long u = u0; u < u1 && ok; ++u) {
-                const long long t = u / KB;
-                const int kb = (int)(u % KB);
-                const int mt = (int)(t / p.n_tiles), nt = (int)(t % p.n_tiles);
+            // unit positions advance by increments (no division per unit)
+            UnitPos up(u0, KB, p.n_tiles);
+            for (long long u = u0; u < u1 && ok; ++u, up.next(KB, p.n_tiles)) {
+                const int kb = up.kb, mt = up.mt, nt = up.nt;
                 if (!wait_bounded(&empty[rs.idx], rs.phase ^ 1u, wc)) { ok = false; break; }
                 mbar_arrive_expect_tx(&full[rs.idx], C::STAGE);
                 uint8_t* st = smem + rs.idx * C::STAGE;

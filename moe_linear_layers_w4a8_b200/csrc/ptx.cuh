@@ -475,6 +475,29 @@ __device__ __forceinline__ bool warp_wait_bounded(uint64_t* bar, uint32_t parity
     return __all_sync(0xFFFFFFFFu, ok) != 0;
 }
 
+// Position (tile t = mt * n_tiles + nt, k-block kb) of a unit, advanced one
+// unit at a time without division.
+struct UnitPos {
+    long long t;
+    int kb, mt, nt;
+    __device__ __forceinline__ UnitPos(long long u, long long KB, int n_tiles) {
+        t = u / KB;
+        kb = (int)(u - t * KB);
+        mt = (int)(t / n_tiles);
+        nt = (int)(t - (long long)mt * n_tiles);
+    }
+    __device__ __forceinline__ void next(long long KB, int n_tiles) {
+        if (++kb == KB) {
+            kb = 0;
+            ++t;
+            if (++nt == n_tiles) {
+                nt = 0;
+                ++mt;
+            }
+        }
+    }
+};
+
 // Position in a ring of n stages and the parity of its current pass.
 struct Ring {
     uint32_t idx = 0, phase = 0;

@@ -18,6 +18,7 @@
 #include "gemm_launch.cuh"
 #include "kernels_misc.cuh"
 #include "gemm_w8a8.cuh"
+#include "gemm_w4a16.cuh"
 
 using namespace w4a8;
 
@@ -371,12 +372,12 @@ struct W8Plan {
     size_t flags_off, ws_bytes;
 };
 
-W8Plan plan_w8(int M, int N, int K, int sms) {
+W8Plan plan_w8(int M, int N, int K, int sms, int kblock = 128) {
     W8Plan pl{};
     pl.bn = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256;
     pl.m_tiles = (M + pl.bn - 1) / pl.bn;
     pl.n_tiles = (N + 127) / 128;
-    pl.KB = K / 128;
+    pl.KB = K / kblock;
     const long long tiles = (long long)pl.m_tiles * pl.n_tiles;
     const long long U = tiles * pl.KB;
     if (sms <= 0) sms = 1;
@@ -450,6 +451,105 @@ w4a8_status w8_gemm_impl(const int8_t* qx, const float* s_x, const int8_t* q_w, 
     p.wait_ns = kDefaultWaitNs;
     return static_cast<w4a8_status>(
         launch_w8a8(pl.bn, pl.split, tw, tx, p, pl.grid, static_cast<cudaStream_t>(stream)));
+}
+
+// W4A16: (tile, k-block of 64) units; the fp32 partial tiles of a split have
+// the int32 ones' size.
+W8Plan plan_w16(int M, int N, int K, int sms) { return plan_w8(M, N, K, sms, 64); }
+
+// 3-D tensor map over bf16 activations [rows][K] (row stride ldx elements)
+// seen as (64 k, row, k-block): box 64 k x box_rows rows x box_kb k-blocks,
+// 128-byte swizzle (the MMA's K-major layout, one 1024-byte-aligned sub-tile
+// per k-block).
+bool make_bf16_k64_tmap(CUtensorMap* map, const void* base, long long rows, int K, int ldx, int box_rows,
+                        int box_kb) {
+    EncodeTiledFn enc = get_encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {64, (cuuint64_t)rows, (cuuint64_t)(K / 64)};
+    cuuint64_t strides[2] = {(cuuint64_t)ldx * 2, 128};
+    cuuint32_t box[3] = {64, (cuuint32_t)box_rows, (cuuint32_t)box_kb};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// 2-D tensor map over a [G][N] matrix of group scales (fp32) or zero-points
+// (uint8), box 128 columns x box_rows groups.
+bool make_group_tmap(CUtensorMap* map, const void* base, int G, int N, bool f32, int box_rows) {
+    EncodeTiledFn enc = get_encode_fn();
+    if (!enc) return false;
+    const int es = f32 ? 4 : 1;
+    cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)G};
+    cuuint64_t strides[1] = {(cuuint64_t)N * es};
+    cuuint32_t box[2] = {128, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+                     const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// k-blocks of 64 per activation box of the W4A16 kernel (about 16 KB).
+int w16_box_kb(int bn) {
+    const int k = 16384 / (bn * 128);
+    return k < 1 ? 1 : (k > 8 ? 8 : k);
+}
+
+w4a8_status w16_gemm_impl(const uint16_t* X, int M, int ldx, const uint8_t* packed, const float* s_w,
+                          const uint8_t* z, const w4a8_wdesc* w, uint16_t* Y, int ldy, void* workspace,
+                          size_t ws_bytes, int32_t* dev_status, void* stream) {
+    w4a8_status st = check_wdesc(w);
+    if (st != W4A8_OK) return st;
+    if (M < 0 || !Y || ldy < w->N) return W4A8_ERR_INVALID_ARG;
+    if (M == 0) return W4A8_OK;
+    if (!X || !packed || !s_w || ldx < w->K) return W4A8_ERR_INVALID_ARG;
+    if (w->symmetric ? (z != nullptr) : (z == nullptr)) return W4A8_ERR_FORMAT_MISMATCH;
+    if (!aligned16(X) || ldx % 8 != 0 || !aligned16(packed) || !aligned16(s_w) || (z && !aligned16(z)))
+        return W4A8_ERR_INVALID_ARG;
+    if (w->K > (1 << 24) || M > (1 << 24)) return W4A8_ERR_UNSUPPORTED_SHAPE;
+    const W8Plan pl = plan_w16(M, w->N, w->K, sm_count_current());
+    if (pl.ws_bytes > 0 && (!workspace || ws_bytes < pl.ws_bytes)) return W4A8_ERR_WORKSPACE;
+    // scale / zero-point rows of one weight stage of 8 k-blocks: 8 groups of
+    // 64, or up to 5 groups of 128 when the stage starts inside a group
+    const int sg_rows = w->group == 64 ? 8 : 5;
+    CUtensorMap tx, ts, tz;
+    if (!make_bf16_k64_tmap(&tx, X, M, w->K, ldx, pl.bn, w16_box_kb(pl.bn)) ||
+        !make_group_tmap(&ts, s_w, w->K / w->group, w->N, true, sg_rows))
+        return W4A8_ERR_CUDA;
+    if (z) {
+        if (!make_group_tmap(&tz, z, w->K / w->group, w->N, false, sg_rows)) return W4A8_ERR_CUDA;
+    } else {
+        tz = ts;  // never read by the symmetric kernels
+    }
+    W16Params p{};
+    p.sg_rows = sg_rows;
+    p.N = w->N;
+    p.K = w->K;
+    p.M = M;
+    p.G = w->K / w->group;
+    p.group = w->group;
+    p.n_tiles = pl.n_tiles;
+    p.m_tiles = pl.m_tiles;
+    p.KB = pl.KB;
+    p.units_per_cta = pl.Q;
+    p.packed = packed;
+    p.s_w = s_w;
+    p.z = z;
+    p.Y = Y;
+    p.ldy = ldy;
+    p.vec16 = (aligned16(Y) && ldy % 8 == 0) ? 1 : 0;
+    p.partial = static_cast<float*>(workspace);
+    p.slots = pl.slots;
+    if (pl.split) {
+        p.flags = reinterpret_cast<unsigned long long*>(static_cast<uint8_t*>(workspace) + pl.flags_off);
+        p.epoch = next_epoch();
+    }
+    p.status = dev_status;
+    p.wait_ns = kDefaultWaitNs;
+    return static_cast<w4a8_status>(launch_w4a16(pl.bn, pl.split, w->symmetric != 0, tx, ts, tz, p, pl.grid,
+                                                 static_cast<cudaStream_t>(stream)));
 }
 
 }  // namespace
@@ -898,6 +998,17 @@ w4a8_status w8a8_pack_weights(const float* W, int K, int N, int8_t* q_w, float* 
 size_t w8a8_gemm_workspace_size(int M, const w4a8_wdesc* w) {
     if (M <= 0 || check_w8desc(w) != W4A8_OK) return 0;
     return plan_w8(M, w->N, w->K, sm_count_current()).ws_bytes;
+}
+
+size_t w4a16_gemm_workspace_size(int M, const w4a8_wdesc* w) {
+    if (M <= 0 || check_wdesc(w) != W4A8_OK) return 0;
+    return plan_w16(M, w->N, w->K, sm_count_current()).ws_bytes;
+}
+
+w4a8_status w4a16_gemm(const uint16_t* X, int M, int ldx, const uint8_t* packed, const float* s_w, const uint8_t* z,
+                       const w4a8_wdesc* w, uint16_t* Y, int ldy, void* workspace, size_t ws_bytes,
+                       int32_t* dev_status, void* stream) {
+    return w16_gemm_impl(X, M, ldx, packed, s_w, z, w, Y, ldy, workspace, ws_bytes, dev_status, stream);
 }
 
 w4a8_status w8a8_gemm(const int8_t* qx, const float* s_x, const int8_t* q_w, const float* s_w, const w4a8_wdesc* w,

@@ -366,3 +366,37 @@ def w8a8_dequant_gemm(qx: np.ndarray, s_x: np.ndarray, qw: np.ndarray, s_w: np.n
     Xd = s_x.astype(np.float64)[:, None] * qx.astype(np.float64)
     Wd = qw.astype(np.float64) * s_w.astype(np.float64)[None, :]
     return Xd @ Wd
+
+
+# --------------------------------------------------------------------------
+# W4A16: weight-only, dequantized inside the GEMM ("Inference Quantization
+# ch.1" §2 and §3.1-3.2: W_fp ~ s_w W_int, Y = X_fp dequant(W_int, s_w))
+# --------------------------------------------------------------------------
+
+def w4a16_dequant_f32(codes: np.ndarray, s: np.ndarray, z, group: int) -> np.ndarray:
+    """The dequantized weight before its bf16 rounding: fp32 [K, N] with
+    w[k, n] = s[g, n] * (q[n, k] - z[g, n]) rounded once to binary32
+    (g = k // group; z = 0 for symmetric codes).  q - z is a small integer,
+    so the only rounding is that of the product."""
+    codes = np.asarray(codes, dtype=np.int8)
+    N, K = codes.shape
+    g = np.arange(K) // group
+    d = codes.T.astype(np.float32)
+    if z is not None:
+        d = d - np.asarray(z, dtype=np.uint8)[g, :].astype(np.float32)
+    sk = np.asarray(s, dtype=np.float32)[g, :]
+    return np.multiply(d, sk, dtype=np.float32)
+
+
+def w4a16_dequant(codes: np.ndarray, s: np.ndarray, z, group: int) -> np.ndarray:
+    """The bf16 operand the weight-only GEMM multiplies: raw bf16 bits [K, N]
+    = round-to-nearest-even of w4a16_dequant_f32."""
+    return f64_to_bf16(w4a16_dequant_f32(codes, s, z, group).astype(np.float64))
+
+
+def w4a16_gemm(X_bf16: np.ndarray, W_hat_bf16: np.ndarray):
+    """Y = X w_hat in binary64 (both operands are bf16 values, every product is
+    exact in binary64).  Returns (Y [M, N], sum of |terms| [M, N])."""
+    X = bf16_to_f32(X_bf16).astype(np.float64)
+    W = bf16_to_f32(W_hat_bf16).astype(np.float64)
+    return X @ W, np.abs(X) @ np.abs(W)

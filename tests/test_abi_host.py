@@ -21,12 +21,13 @@ def lib():
 def _declared_functions():
     src = open(os.path.join(ROOT, "include", "w4a8.h")).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(w4a8_[a-z0-9_]+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b((?:w4a8|w8a8|w4a16)_[a-z0-9_]+)\s*\(", src)))
 
 
 def test_header_declares_the_boundary_calls():
     names = _declared_functions()
-    for required in ("w4a8_pack_weights", "w4a8_quant_act", "w4a8_gemm", "w4a8_moe_grouped_gemm"):
+    for required in ("w4a8_pack_weights", "w4a8_quant_act", "w4a8_gemm", "w4a8_moe_grouped_gemm",
+                     "w8a8_gemm", "w4a16_gemm"):
         assert required in names
 
 
@@ -40,7 +41,7 @@ def test_library_exports_nothing_else(lib):
     from moe_linear_layers_w4a8_b200 import library_path
     out = subprocess.run(["nm", "-D", "--defined-only", library_path()], capture_output=True, text=True).stdout
     exported = {l.split()[-1] for l in out.splitlines() if " T " in l}
-    ours = {n for n in exported if n.startswith("w4a8_")}
+    ours = {n for n in exported if n.startswith(("w4a8_", "w8a8_", "w4a16_"))}
     assert ours == set(_declared_functions())
 
 
@@ -121,6 +122,37 @@ def test_linear_sizes_and_rejections(lib):
     assert lib.w4a8_linear(FAKE, 16, 512, FAKE, FAKE, None, ctypes.byref(d), FAKE, 100, FAKE, need, None, None) == 1
     assert lib.w4a8_linear(FAKE, -1, 512, FAKE, FAKE, None, ctypes.byref(d), FAKE, 512, FAKE, need, None, None) == 1
     assert lib.w4a8_linear(FAKE, 0, 512, FAKE, FAKE, None, ctypes.byref(d), FAKE, 512, FAKE, 0, None, None) == 0
+
+
+def test_w4a16_sizes_and_rejections(lib):
+    d = _desc()
+    need = lib.w4a16_gemm_workspace_size(16, ctypes.byref(d))
+    # split-K partials only when the tiles leave SMs idle: with no GPU to ask
+    # the SM count is taken as 1 and the plan needs no workspace
+    assert lib.w4a16_gemm_workspace_size(0, ctypes.byref(d)) == 0
+    bad = _desc(layout_version=2)
+    assert lib.w4a16_gemm_workspace_size(16, ctypes.byref(bad)) == 0
+    args = lambda **k: dict(dict(X=FAKE, M=16, ldx=512, z=None, d=d, ldy=512, ws=FAKE, wsb=need), **k)
+
+    def call(**k):
+        a = args(**k)
+        return lib.w4a16_gemm(a["X"], a["M"], a["ldx"], FAKE, FAKE, a["z"], ctypes.byref(a["d"]) if a["d"] else None,
+                              FAKE, a["ldy"], a["ws"], a["wsb"], None, None)
+    assert call(d=bad) == 3
+    assert call(z=FAKE) == 3                               # symmetric weight with zero-points
+    assert call(d=_desc(symmetric=0)) == 3                 # asymmetric weight without them
+    assert call(d=_desc(bits=8)) == 3
+    assert call(M=-1) == 1
+    assert call(ldy=100) == 1
+    assert call(ldx=500) == 1                              # ldx < K
+    assert call(ldx=516) == 1                              # row stride not a multiple of 16 bytes
+    assert call(X=None) == 1
+    assert call(X=ctypes.c_void_p(264)) == 1               # not 16-byte aligned
+    if need > 0:
+        assert call(wsb=need - 1) == 7
+        assert call(ws=None, wsb=0) == 7
+    assert call(M=0) == 0
+    assert call(d=_desc(K=1 << 25, N=64), ldx=1 << 25) == 2
 
 
 def test_pack_rejects_bad_args(lib):

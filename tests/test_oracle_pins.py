@@ -514,3 +514,86 @@ def test_w8a8_integer_sum_brute_force():
     for m in range(3):
         for n in range(4):
             assert acc[m, n] == sum(int(qx[m, k]) * int(qw[k, n]) for k in range(20))
+
+
+# ------------------------------------------------------- W4A16 weight-only --
+
+def test_w4a16_dequant_worked_example_linear_s2(orc, golden):
+    """§2 dequantizes the worked example's codes as s_w * W_int; the weight-only
+    dequant (codes as one column, one group) gives the printed values before
+    its bf16 rounding, and its bf16 rounding is within half a bf16 ulp."""
+    g = golden("lin_s2_worked_int8.txt")
+    codes = np.array([[int(v) for v in g["codes"]]], np.int8)          # [N=1, K=4]
+    s = np.array([[np.float32(0.8) / np.float32(127.0)]], np.float32)    # [G=1, N=1]
+    w32 = orc.w4a16_dequant_f32(codes, s, None, 4)[:, 0]
+    # the page prints its values from the rounded scale 0.0063, so the exact
+    # scale's values agree with them to the printed precision
+    printed = np.array([float(v) for v in g["dequant_printed"]])
+    assert np.all(np.abs(w32.astype(np.float64) - printed) <= 1e-3)
+    assert np.array_equal(w32, codes[0].astype(np.float32) * s[0, 0])
+    wb = orc.bf16_to_f32(orc.w4a16_dequant(codes, s, None, 4))[:, 0].astype(np.float64)
+    assert np.all(np.abs(wb - w32) <= np.abs(w32) * 2.0 ** -8)  # half a bf16 ulp
+
+
+def test_w4a16_dequant_by_hand_asymmetric_groups():
+    """Asymmetric, group 2, K = 4: q = [0, 15, 7, 8], z = [7, 8], s = [0.5, 0.25]
+    -> s (q - z) = [-3.5, 4.0, -0.25, 0.0] (all exact in bf16); the group
+    index follows k, never the column."""
+    import oracle as O
+    codes = np.array([[0, 15, 7, 8], [8, 7, 15, 0]], np.int8)           # [N=2, K=4]
+    z = np.array([[7, 8], [8, 7]], np.uint8)                             # [G=2, N=2]
+    s = np.array([[0.5, 1.0], [0.25, 2.0]], np.float32)
+    w = O.bf16_to_f32(O.w4a16_dequant(codes, s, z, 2)).astype(np.float64)
+    assert w[:, 0].tolist() == [-3.5, 4.0, -0.25, 0.0]
+    # column 1: s = 1 on k 0-1, 2 on k 2-3; q - z = [0, -1, 8, -7]
+    assert w[:, 1].tolist() == [0.0, -1.0, 16.0, -14.0]
+
+
+def test_w4a16_dequant_rounds_the_fp32_product_then_to_bf16():
+    """The reading: one binary32 product, then bf16.  s = 0x3F95AAAB
+    (1.16927087306976318359375), q - z = 3: the exact product is
+    3.5078125 + 2^-23, a binary32 tie that rounds to even, 3.5078125; that
+    is the bf16 midpoint of 3.5 and 3.515625, which rounds to even: 3.5
+    (0x4060).  Rounding the exact product straight to bf16 would give
+    3.515625 (0x4061)."""
+    import oracle as O
+    s = np.array([0x3F95AAAB], np.uint32).view(np.float32).reshape(1, 1)
+    codes = np.array([[3]], np.int8)
+    assert float(O.w4a16_dequant_f32(codes, s, None, 1)[0, 0]) == 3.5078125
+    assert int(O.w4a16_dequant(codes, s, None, 1)[0, 0]) == 0x4060
+
+
+def test_w4a16_gemm_by_hand_and_zero_codes():
+    """Y = X w_hat: X = [1, 2, -1, 0.5] against the column [-3.5, 4, -0.25, 0]
+    gives -3.5 + 8 + 0.25 = 4.75; codes equal to their zero-points give 0."""
+    import oracle as O
+    codes = np.array([[0, 15, 7, 8]], np.int8)
+    z = np.array([[7], [8]], np.uint8)
+    s = np.array([[0.5], [0.25]], np.float32)
+    Wh = O.w4a16_dequant(codes, s, z, 2)
+    X = O.f64_to_bf16(np.array([[1.0, 2.0, -1.0, 0.5]]))
+    Y, A = O.w4a16_gemm(X, Wh)
+    assert Y[0, 0] == 4.75 and A[0, 0] == 3.5 + 8.0 + 0.25
+    Wz = O.w4a16_dequant(np.array([[7, 7, 8, 8]], np.int8), s, z, 2)
+    assert not O.w4a16_gemm(X, Wz)[0].any()
+
+
+def test_w4a16_within_bf16_rounding_of_the_exact_dequant():
+    """The weight-only product differs from X times the exact dequantized
+    weight (the W4A8 oracle's binary64 s (q - z)) only by the weights' bf16
+    rounding: |Y - Y_exact| <= 2^-8 sum |x| |w| (fp32 then bf16 rounding,
+    each at most half an ulp)."""
+    import oracle as O
+    rng = np.random.default_rng(6)
+    K, N = 256, 64
+    W = (rng.standard_normal((K, N)) * 0.02).astype(np.float32)
+    for sym in (True, False):
+        codes, s, z, _ = O.quant_weights(W, 64, sym)
+        zz = None if sym else z
+        Wh = O.w4a16_dequant(codes, s, zz, 64)
+        Wx = O.dequant_weights(codes, s, zz, 64)                    # binary64 [K, N]
+        X = O.f64_to_bf16(rng.standard_normal((5, K)))
+        Xf = O.bf16_to_f32(X).astype(np.float64)
+        Y, _ = O.w4a16_gemm(X, Wh)
+        Yx = Xf @ Wx
+        assert np.all(np.abs(Y - Yx) <= 2.0 ** -8 * (np.abs(Xf) @ np.abs(Wx)) + 1e-30)
