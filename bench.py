@@ -56,7 +56,7 @@ L2_BYTES = 126 * 1024 * 1024
 
 DEFAULT_STEPS = {"decode": 20000, "prefill": 1500, "moe_sym": 2000, "moe_asym_decode": 400,
                  "moe_asym_prefill": 200, "w8a8_decode": 20000, "w8a8_prefill": 1500,
-                 "w4a16_decode": 20000, "w4a16_prefill": 1500}
+                 "w4a16_decode": 20000, "w4a16_prefill": 1500, "moe_asym_prefill_e32": 400}
 
 
 # ---------------------------------------------------------------- peaks ---
@@ -240,17 +240,20 @@ class LinearWorkload:
 
     def kernel_roofline(self, peaks):
         M, K, N, g = self.M, self.K, self.N, self.group
+        kname = ("w8a8_gemm_kernel" if self.w8 else "w4a16_gemm_kernel" if self.w16 else
+                 "w4a8_gemm_tc_kernel")
         if self.decode:
             # weights + scales, activations (int8 + s_x, or bf16), bf16 output
             alg = self.w_bytes + (2 * M * K if self.w16 else M * K + 4 * M) + 2 * M * N
             return dict(bound="hbm", per_launch=alg, unit="GB/s", scale=1e9, peak=peaks["hbm"],
-                        peak_note=f"hbm_gbs ({peaks['source']})")
+                        peak_note=f"hbm_gbs ({peaks['source']})", kernel_name=kname)
         ops = 2.0 * M * N * K
         if self.w16:
             return dict(bound="tensor", per_launch=ops, unit="TFLOP/s", scale=1e12, peak=peaks["bf16_sus"],
-                        peak_note=f"bf16_tflops_sustained ({peaks['source']})")
+                        peak_note=f"bf16_tflops_sustained ({peaks['source']})", kernel_name=kname)
         return dict(bound="tensor", per_launch=ops, unit="TOPS", scale=1e12, peak=2.0 * peaks["bf16_sus"],
-                    peak_note=f"2 x bf16_tflops_sustained ({peaks['source']}; int8/bf16 nominal ratio 2)")
+                    peak_note=f"2 x bf16_tflops_sustained ({peaks['source']}; int8/bf16 nominal ratio 2)",
+                    kernel_name=kname)
 
     def config(self):
         wfmt = ("per-channel int8 weights (W8A8)" if self.w8 else
@@ -800,7 +803,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="decode",
                     choices=["decode", "prefill", "moe_sym", "moe_asym_decode", "moe_asym_prefill", "w8a8_decode",
-                             "w8a8_prefill", "w4a16_decode", "w4a16_prefill"])
+                             "w8a8_prefill", "w4a16_decode", "w4a16_prefill", "moe_asym_prefill_e32"])
     ap.add_argument("--m", type=int, default=None, help="rows of the linear workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--main-only", action="store_true",

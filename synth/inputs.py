@@ -50,6 +50,11 @@ CONFIGS = {
                             symmetric=False, zipf=1.1, w_outlier_p=0.001, seed=0),
     "moe_asym_prefill": dict(T=8192, H=7168, E=256, topk=8, I=2048, group=64,
                              symmetric=False, zipf=1.1, w_outlier_p=0.001, seed=0),
+    # the asymmetric prefill layer scaled down for counter captures: the same
+    # shapes per expert and the same mean rows per expert (T * topk / E = 256)
+    # with 1/8 of the experts and tokens (about 0.7 GB of packed weights)
+    "moe_asym_prefill_e32": dict(T=1024, H=7168, E=32, topk=8, I=2048, group=64,
+                                 symmetric=False, zipf=1.1, w_outlier_p=0.001, seed=0),
 }
 
 
