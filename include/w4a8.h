@@ -177,6 +177,13 @@ W4A8_API w4a8_status w4a8_quant_act(const uint16_t* X, int M, int K, int ldx, in
  *         launch that ended with W4A8_ERR_TIMEOUT, zero the workspace before
  *         replaying a captured graph of that launch (a replay repeats the
  *         epoch).  Calls that can overlap on the GPU need separate workspaces.
+ * Co-residency: the split-K schedule launches at most one CTA per SM and the
+ *         CTA that sums a tile waits for flags set by later CTAs of the same
+ *         grid, so it assumes the whole grid is resident at once.  When other
+ *         work holds SMs for longer than the wait limit (4 s) the call ends
+ *         with W4A8_ERR_TIMEOUT in dev_status instead of a result (no hang).
+ *         The same holds for the split-K schedules of w8a8_gemm and
+ *         w4a16_gemm.
  * Errors: INVALID_ARG, FORMAT_MISMATCH (bad descriptor), WORKSPACE,
  *         UNSUPPORTED_SHAPE; TIMEOUT via dev_status.
  */

@@ -221,21 +221,45 @@ __device__ __forceinline__ void tile_blocks(const GemmParams& p, int nt, int& nb
     }
 }
 
-// Work range of this CTA in (tile, group) units.
+// Work range of this CTA in (tile, group) units.  SplitK: a contiguous run
+// of units (a tile may be shared by several CTAs).  The other modes hand out
+// whole tiles round-robin: the CTA's i-th tile is blockIdx.x + i * gridDim.x,
+// so the CTAs running at the same time work on neighbouring tiles (the same
+// token block and the same expert's weights), and a tile's operands are
+// fetched from HBM about once and shared through L2.  The range stays
+// contiguous in a virtual numbering (the CTA's i-th tile is virtual tile
+// blockIdx.x * waves + i); tile_of() maps a virtual tile to the real one.
 template <int MODE>
 __device__ __forceinline__ void cta_units(const GemmParams& p, long long& u0, long long& u1, long long& Q) {
-    long long U;
-    if constexpr (MODE == kModeGateUp || MODE == kModeDown) {
-        const long long tiles = (long long)__ldg(p.mtile_off + p.E) * p.n_tiles;
-        U = tiles * p.G;
-        Q = (long long)p.G * ((tiles + gridDim.x - 1) / gridDim.x);
-    } else {
-        U = (long long)p.m_tiles * p.n_tiles * p.G;
+    if constexpr (MODE == kModeSplitK) {
+        const long long U = (long long)p.m_tiles * p.n_tiles * p.G;
         Q = p.units_per_cta;
+        u0 = (long long)blockIdx.x * Q;
+        u1 = min(u0 + Q, U);
+        if (u0 > U) u0 = U;
+    } else {
+        long long tiles;
+        if constexpr (MODE == kModeGateUp || MODE == kModeDown)
+            tiles = (long long)__ldg(p.mtile_off + p.E) * p.n_tiles;
+        else
+            tiles = (long long)p.m_tiles * p.n_tiles;
+        const long long grid = gridDim.x;
+        const long long waves = (tiles + grid - 1) / grid;
+        const long long mine = (long long)blockIdx.x < tiles ? (tiles - 1 - blockIdx.x) / grid + 1 : 0;
+        Q = (long long)p.G * waves;
+        u0 = (long long)blockIdx.x * Q;
+        u1 = u0 + mine * p.G;
     }
-    u0 = (long long)blockIdx.x * Q;
-    u1 = min(u0 + Q, U);
-    if (u0 > U) u0 = U;
+}
+
+template <int MODE>
+__device__ __forceinline__ long long tile_of(long long t_virtual, long long Q, int G) {
+    if constexpr (MODE == kModeSplitK) {
+        return t_virtual;
+    } else {
+        const long long waves = Q / G;
+        return (long long)blockIdx.x + (t_virtual - (long long)blockIdx.x * waves) * gridDim.x;
+    }
 }
 
 constexpr int kUnpackWarps = 4;
@@ -388,7 +412,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             bool ok = true;
             for (long long u = u0; u < u1 && ok;) {
                 const Segment sg = segment_at(u, u1, G);
-                const TileInfo ti = decode_tile<BN, MODE>(p, sg.t);
+                const TileInfo ti = decode_tile<BN, MODE>(p, tile_of<MODE>(sg.t, Q, G));
                 int nb0, nb1;
                 tile_blocks<MODE>(p, ti.nt, nb0, nb1);
                 const uint8_t* wbase = p.packed + (long long)ti.e * p.packed_estride;
@@ -434,7 +458,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             bool ok = true;
             for (long long u = u0; u < u1 && ok;) {
                 const Segment sg = segment_at(u, u1, G);
-                const TileInfo ti = decode_tile<BN, MODE>(p, sg.t);
+                const TileInfo ti = decode_tile<BN, MODE>(p, tile_of<MODE>(sg.t, Q, G));
                 int nb0, nb1;
                 tile_blocks<MODE>(p, ti.nt, nb0, nb1);
                 const int wrow = ti.e * G;
@@ -636,7 +660,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const Segment sg = segment_at(u, u1, G);
             const long long t = sg.t;
             const int gb = sg.gb, ge = sg.ge;
-            const TileInfo ti = decode_tile<BN, MODE>(p, t);
+            const TileInfo ti = decode_tile<BN, MODE>(p, tile_of<MODE>(t, Q, G));
             int nb0, nb1;
             tile_blocks<MODE>(p, ti.nt, nb0, nb1);
             const bool n_valid = (half == 0) || (nb1 >= 0);

@@ -254,10 +254,13 @@ __global__ void __launch_bounds__(kW16Threads, 1)
 
     const long long KB = p.KB;
     const int KBi = p.KB;
-    const long long U = (long long)p.m_tiles * p.n_tiles * KB;
-    const long long Q = p.units_per_cta;
-    const long long u0 = min((long long)blockIdx.x * Q, U);
-    const long long u1 = min(u0 + Q, U);
+    const long long tiles = (long long)p.m_tiles * p.n_tiles;
+    const long long U = tiles * KB;
+    // split-K: contiguous unit ranges; otherwise whole tiles round-robin
+    const RoundRobin rrt(tiles, KB);
+    const long long Q = SPLIT ? p.units_per_cta : rrt.waves * KB;
+    const long long u0 = SPLIT ? min((long long)blockIdx.x * Q, U) : rrt.u0;
+    const long long u1 = SPLIT ? min(u0 + Q, U) : rrt.u1;
     const int kb_shift = p.group == 128 ? 1 : 0;   // k-blocks of 64 per group: 1 << kb_shift
 
     if (warp == 0) {
@@ -268,7 +271,8 @@ __global__ void __launch_bounds__(kW16Threads, 1)
             bool ok = true;
             // positions advance by increments: one 64-bit division per unit
             // would cost more than the copies it schedules
-            UnitPos up(u0, KB, p.n_tiles);
+            UnitPos up = SPLIT ? UnitPos(u0, KB, p.n_tiles)
+                               : UnitPos(u0, KB, p.n_tiles, rrt.v0, blockIdx.x, gridDim.x);
             for (long long u = u0; u < u1 && ok;) {
                 const int kb = up.kb, nt = up.nt;
                 const int len = (int)min((long long)min(kW16KSW, KBi - kb), u1 - u);
@@ -307,7 +311,8 @@ __global__ void __launch_bounds__(kW16Threads, 1)
             Ring rx;
             long long issued = 0;
             bool ok = true;
-            UnitPos up(u0, KB, p.n_tiles);
+            UnitPos up = SPLIT ? UnitPos(u0, KB, p.n_tiles)
+                               : UnitPos(u0, KB, p.n_tiles, rrt.v0, blockIdx.x, gridDim.x);
             // activations may come from the kernel launched just before
             pdl_wait_prerequisites();
             for (long long u = u0; u < u1 && ok;) {
@@ -405,7 +410,8 @@ __global__ void __launch_bounds__(kW16Threads, 1)
         int g0 = 0, g_prev = -1;
         uint64_t A[5], S[5];
         bool ok = true;
-        UnitPos up(u0, KB, p.n_tiles);
+        UnitPos up = SPLIT ? UnitPos(u0, KB, p.n_tiles)
+                               : UnitPos(u0, KB, p.n_tiles, rrt.v0, blockIdx.x, gridDim.x);
         for (long long u = u0; u < u1;) {
             const int kb = up.kb;
             const int len = (int)min((long long)min(C::KA, KBi - kb), u1 - u);
@@ -492,7 +498,8 @@ __global__ void __launch_bounds__(kW16Threads, 1)
             const int kb0 = (int)(u % KB);
             const long long seg_end = min(u1, (t + 1) * KB);
             const int kb1 = (int)(seg_end - t * KB);
-            const int mt = (int)(t / p.n_tiles), nt = (int)(t % p.n_tiles);
+            const long long ta = SPLIT ? t : rrt.tile(t);
+            const int mt = (int)(ta / p.n_tiles), nt = (int)(ta % p.n_tiles);
             const int row0 = mt * BN;
             const int rows_valid = min(BN, p.M - row0);
             const int ncols = min(128, p.N - nt * 128);

@@ -122,10 +122,13 @@ __global__ void __launch_bounds__(kW8Threads, 1)
     const WaitCtx wc{abort_flag, p.status, wait_cycles_for_ns(p.wait_ns)};
 
     const long long KB = p.KB;
-    const long long U = (long long)p.m_tiles * p.n_tiles * KB;
-    const long long Q = p.units_per_cta;
-    const long long u0 = min((long long)blockIdx.x * Q, U);
-    const long long u1 = min(u0 + Q, U);
+    const long long tiles = (long long)p.m_tiles * p.n_tiles;
+    const long long U = tiles * KB;
+    // split-K: contiguous unit ranges; otherwise whole tiles round-robin
+    const RoundRobin rrt(tiles, KB);
+    const long long Q = SPLIT ? p.units_per_cta : rrt.waves * KB;
+    const long long u0 = SPLIT ? min((long long)blockIdx.x * Q, U) : rrt.u0;
+    const long long u1 = SPLIT ? min(u0 + Q, U) : rrt.u1;
 
     if (warp == 0) {
         // ------------------------------------------------------- producer --
@@ -135,7 +138,8 @@ __global__ void __launch_bounds__(kW8Threads, 1)
             bool ok = true;
             bool waited = false;
             // unit positions advance by increments (no division per unit)
-            UnitPos up(u0, KB, p.n_tiles);
+            UnitPos up = SPLIT ? UnitPos(u0, KB, p.n_tiles)
+                               : UnitPos(u0, KB, p.n_tiles, rrt.v0, blockIdx.x, gridDim.x);
             for (long long u = u0; u < u1 && ok; ++u, up.next(KB, p.n_tiles)) {
                 const int kb = up.kb, mt = up.mt, nt = up.nt;
                 if (!wait_bounded(&empty[rs.idx], rs.phase ^ 1u, wc)) { ok = false; break; }
@@ -210,7 +214,8 @@ __global__ void __launch_bounds__(kW8Threads, 1)
             const int kb0 = (int)(u % KB);
             const long long seg_end = min(u1, (t + 1) * KB);
             const int kb1 = (int)(seg_end - t * KB);
-            const int mt = (int)(t / p.n_tiles), nt = (int)(t % p.n_tiles);
+            const long long ta = SPLIT ? t : rrt.tile(t);
+            const int mt = (int)(ta / p.n_tiles), nt = (int)(ta % p.n_tiles);
             const int n = nt * 128 + r;
             const int row0 = mt * BN;
             const int rows_valid = min(BN, p.M - row0);

@@ -475,26 +475,59 @@ __device__ __forceinline__ bool warp_wait_bounded(uint64_t* bar, uint32_t parity
     return __all_sync(0xFFFFFFFFu, ok) != 0;
 }
 
-// Position (tile t = mt * n_tiles + nt, k-block kb) of a unit, advanced one
-// unit at a time without division.
+// Position of a unit: k-block kb of the virtual tile t, which is the real
+// tile ta = base + (t - v0) * stride (stride 1, base = v0 = 0 for a
+// contiguous range; stride = the grid size for tiles handed out round-robin),
+// ta = mt * n_tiles + nt.  Advanced one unit at a time: no division per
+// unit, one per tile when tiles are strided.
 struct UnitPos {
-    long long t;
+    long long t, ta, stride;
     int kb, mt, nt;
-    __device__ __forceinline__ UnitPos(long long u, long long KB, int n_tiles) {
+    __device__ __forceinline__ UnitPos(long long u, long long KB, int n_tiles, long long v0 = 0, long long base = 0,
+                                       long long stride_ = 1) {
         t = u / KB;
         kb = (int)(u - t * KB);
-        mt = (int)(t / n_tiles);
-        nt = (int)(t - (long long)mt * n_tiles);
+        stride = stride_;
+        ta = base + (t - v0) * stride;
+        mt = (int)(ta / n_tiles);
+        nt = (int)(ta - (long long)mt * n_tiles);
     }
     __device__ __forceinline__ void next(long long KB, int n_tiles) {
         if (++kb == KB) {
             kb = 0;
             ++t;
-            if (++nt == n_tiles) {
-                nt = 0;
-                ++mt;
+            ta += stride;
+            if (stride == 1) {
+                if (++nt == n_tiles) {
+                    nt = 0;
+                    ++mt;
+                }
+            } else {
+                mt = (int)(ta / n_tiles);
+                nt = (int)(ta - (long long)mt * n_tiles);
             }
         }
+    }
+};
+
+// Whole tiles handed out round-robin (the CTA's i-th tile is blockIdx.x + i *
+// gridDim.x), kept as a contiguous range of units in a virtual tile numbering
+// (the CTA's i-th tile is virtual tile blockIdx.x * waves + i): CTAs running
+// at the same time then work on neighbouring tiles and share their operands
+// through L2.
+struct RoundRobin {
+    long long waves, v0, u0, u1;
+    __device__ __forceinline__ RoundRobin(long long tiles, long long KB) {
+        const long long grid = gridDim.x, c = blockIdx.x;
+        waves = (tiles + grid - 1) / grid;
+        const long long mine = c < tiles ? (tiles - 1 - c) / grid + 1 : 0;
+        v0 = c * waves;
+        u0 = v0 * KB;
+        u1 = u0 + mine * KB;
+    }
+    // real tile of virtual tile t
+    __device__ __forceinline__ long long tile(long long t) const {
+        return (long long)blockIdx.x + (t - v0) * (long long)gridDim.x;
     }
 };
 
