@@ -96,9 +96,10 @@ def _rank_main(rank, world, port, sym, out):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("sym", [True, False])
-def test_two_ranks_equal_one_process_layer(sym):
-    world = 2
+@pytest.mark.parametrize("world,sym", [(2, True), (2, False), (4, True)])
+def test_ranks_equal_one_process_layer(world, sym):
+    """2 and 4 ranks (4 experts / 2 experts per rank): every rank's output
+    equals the one-process layer on its tokens, and rows really travel."""
     port = _free_port()
     with mp.Manager() as mgr:
         out = mgr.dict()
