@@ -226,7 +226,7 @@ class LinearWorkload:
         return statistics.mean(times), None
 
     def release(self):
-        for a in ("copies", "X", "q", "s", "Y", "ws", "lws", "X_dev2", "Y_pin", "X_pin"):
+        for a in ("copies", "X", "q", "s", "Y", "ws", "lws", "X_dev2", "Y_pin", "X_pin", "Y2", "lws2"):
             if hasattr(self, a):
                 delattr(self, a)
 
@@ -273,14 +273,18 @@ class LinearWorkload:
     def e2e_setup(self):
         import torch
         self.X_pin = self.X_host.pin_memory()
-        self.Y_pin = torch.empty(self.M, self.N, dtype=torch.bfloat16).pin_memory()
-        self.X_dev2 = torch.empty_like(self.X)
-        return self.X_pin.numel() * 2, self.Y_pin.numel() * 2
+        # two steps in flight (one per stream), each with its own buffers
+        self.Y_pin = [torch.empty(self.M, self.N, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+        self.X_dev2 = [torch.empty_like(self.X) for _ in range(2)]
+        self.Y2 = [torch.empty_like(self.Y) for _ in range(2)]
+        self.lws2 = [torch.empty_like(self.lws) for _ in range(2)]
+        return self.X_pin.numel() * 2, self.Y_pin[0].numel() * 2
 
     def e2e_step(self, i):
-        self.X_dev2.copy_(self.X_pin, non_blocking=True)
-        Y = self._linear(self.X_dev2, self.copies[i % len(self.copies)], out=self.Y, workspace=self.lws)
-        self.Y_pin.copy_(Y, non_blocking=True)
+        b = i % 2
+        self.X_dev2[b].copy_(self.X_pin, non_blocking=True)
+        Y = self._linear(self.X_dev2[b], self.copies[i % len(self.copies)], out=self.Y2[b], workspace=self.lws2[b])
+        self.Y_pin[b].copy_(Y, non_blocking=True)
 
     # CPU oracle on a bounded sample of the same workload
     def oracle_step_setup(self, n_cols):
@@ -375,7 +379,7 @@ class MoEWorkload:
         return stage_ms["gate_up"], stage_ms
 
     def release(self):
-        for a in ("w1", "w2", "ws", "out", "X", "L", "X2", "L2", "out_pin", "X_pin", "L_pin"):
+        for a in ("w1", "w2", "ws", "out", "X", "L", "X2", "L2", "out_pin", "X_pin", "L_pin", "out2", "ws2"):
             if hasattr(self, a):
                 delattr(self, a)
 
@@ -410,17 +414,21 @@ class MoEWorkload:
         import torch
         self.X_pin = self.X_host.pin_memory()
         self.L_pin = self.L_host.pin_memory()
-        self.out_pin = torch.empty(self.T, self.H, dtype=torch.bfloat16).pin_memory()
-        self.X2 = torch.empty_like(self.X)
-        self.L2 = torch.empty_like(self.L)
-        return self.X_pin.numel() * 2 + self.L_pin.numel() * 4, self.out_pin.numel() * 2
+        # two steps in flight (one per stream), each with its own buffers
+        self.out_pin = [torch.empty(self.T, self.H, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+        self.X2 = [torch.empty_like(self.X) for _ in range(2)]
+        self.L2 = [torch.empty_like(self.L) for _ in range(2)]
+        self.out2 = [torch.empty_like(self.out) for _ in range(2)]
+        self.ws2 = [torch.empty_like(self.ws) for _ in range(2)]
+        return self.X_pin.numel() * 2 + self.L_pin.numel() * 4, self.out_pin[0].numel() * 2
 
     def e2e_step(self, i):
-        self.X2.copy_(self.X_pin, non_blocking=True)
-        self.L2.copy_(self.L_pin, non_blocking=True)
-        r = self.m.w4a8_moe_grouped_gemm(self.X2, self.L2, self.topk, self.w1, self.w2, workspace=self.ws,
-                                         out=self.out)
-        self.out_pin.copy_(r["out"], non_blocking=True)
+        b = i % 2
+        self.X2[b].copy_(self.X_pin, non_blocking=True)
+        self.L2[b].copy_(self.L_pin, non_blocking=True)
+        r = self.m.w4a8_moe_grouped_gemm(self.X2[b], self.L2[b], self.topk, self.w1, self.w2, workspace=self.ws2[b],
+                                         out=self.out2[b])
+        self.out_pin[b].copy_(r["out"], non_blocking=True)
 
     def oracle_step_setup(self, n_tokens):
         import numpy as np
@@ -588,17 +596,35 @@ def measure(args, wl, K, W, peaks, world, rank, local, cpu_budget_s):
     if stage_ms is not None:
         roofline["stage_ms"] = {k: round(v, 5) for k, v in stage_ms.items()}
 
-    # end to end through the public API with host buffers
+    # end to end through the public API with host buffers: every step copies
+    # its input from pinned host memory and its result back; consecutive steps
+    # alternate between two streams (own buffers and workspace each), so one
+    # step's copies overlap the other's kernels, as a serving loop would run them
     h2d, d2h = wl.e2e_setup()
     Ke = max(1, min(K, 2000 if wl.name == "decode" else max(10, K // 4)))
-    for i in range(min(W, 20)):
-        wl.e2e_step(i)
+    main = torch.cuda.current_stream()
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+
+    def run_e2e(first, n):
+        for i in range(first, first + n):
+            with torch.cuda.stream(streams[i % 2]):
+                wl.e2e_step(i)
+
+    for st in streams:
+        st.wait_stream(main)
+    run_e2e(0, min(W, 20))
+    for st in streams:
+        main.wait_stream(st)
+    torch.cuda.synchronize()
     barrier_sync(torch, world)
     s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s2.record()
-    for i in range(Ke):
-        wl.e2e_step(i)
-    e2.record()
+    s2.record(main)
+    for st in streams:
+        st.wait_stream(main)
+    run_e2e(0, Ke)
+    for st in streams:
+        main.wait_stream(st)
+    e2.record(main)
     torch.cuda.synchronize()
     te = max_over_ranks(torch, world, s2.elapsed_time(e2))
     e2e_value = job_throughput(unit_scale, Ke, world, te)
