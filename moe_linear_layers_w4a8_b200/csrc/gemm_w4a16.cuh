@@ -133,12 +133,6 @@ struct W16Cfg {
     static_assert(SMEM <= 227 * 1024, "shared memory");
 };
 
-__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
-    uint64_t d;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-
 // (w & mask) ^ flip, with the exponent bits of 2^23 set: lop3 with the table
 // of  b ? (a ^ c) : c  (mask in b, flip | 0x4B000000 in c).
 __device__ __forceinline__ uint32_t magic_nibble(uint32_t w, uint32_t mask, uint32_t fc) {

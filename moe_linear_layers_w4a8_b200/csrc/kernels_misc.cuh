@@ -12,6 +12,64 @@ namespace w4a8 {
 
 constexpr int kStatusNonfinite = 4;
 
+// Per-half maximum of the bf16 magnitudes in w and acc (bf16 bits in each
+// 16-bit half).  Unsigned order of the magnitude bits is the order of the
+// magnitudes, and every Inf / NaN pattern (>= 0x7F80) sorts above every
+// finite value, so the row maximum also tells whether the row is finite.
+__device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t acc, uint32_t w) {
+    uint32_t d;
+    asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(acc), "r"(w & 0x7FFF7FFFu));
+    return d;
+}
+
+// The INT8 codes of one 16-byte chunk (8 bf16 values x, k order) for the
+// divisor d (r = the correctly rounded 1 / d), four codes per output word,
+// with the decisions of rne_quotient: the code is RNE(x * r) unless x * r lies
+// within 2^-14 of a half-integer (or is not finite), where the correctly
+// rounded quotient x / d decides.  RNE(x * r) comes from one addition of
+// 1.5 * 2^23: the float grid there is the integers, so the sum is
+// 1.5 * 2^23 + RNE(x * r) exactly and its low byte is the code in two's
+// complement (|x| <= max|x| keeps the code within [-127, 127]).  The
+// distance to the nearest integer, x * r - RNE(x * r), is exact.
+// csum (may be null) receives the sum of the eight codes.
+__device__ __forceinline__ void quant_chunk8(const uint4 raw, float d, float r, uint32_t& q0, uint32_t& q1,
+                                             int32_t* csum) {
+    constexpr float kM = 12582912.0f;  // 1.5 * 2^23
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+    const uint64_t r2 = f2_splat(r), m2 = f2_splat(kM);
+    uint32_t a[8];
+    bool slow = false;
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+        const uint64_t x2 = f2_from_bits(w[h] << 16, w[h] & 0xFFFF0000u);  // (k even, k odd)
+        const uint64_t t2 = f2_mul(x2, r2);
+        const uint64_t a2 = f2_add(t2, m2);
+        const uint64_t e2 = f2_sub(t2, f2_sub(a2, m2));
+        float e0, e1;
+        f2_split(e2, e0, e1);
+        slow |= !(fabsf(e0) < 0.49993896484375f) | !(fabsf(e1) < 0.49993896484375f);  // 0.5 - 2^-14
+        float f0, f1;
+        f2_split(a2, f0, f1);
+        a[2 * h] = __float_as_uint(f0);
+        a[2 * h + 1] = __float_as_uint(f1);
+    }
+    q0 = __byte_perm(__byte_perm(a[0], a[1], 0x0040), __byte_perm(a[2], a[3], 0x0040), 0x5410);
+    q1 = __byte_perm(__byte_perm(a[4], a[5], 0x0040), __byte_perm(a[6], a[7], 0x0040), 0x5410);
+    if (slow) {
+        uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const uint32_t bits = (e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xFFFFu);
+            float t = rne_quotient(bf16_bits_to_f32(bits), d, r);
+            t = fminf(fmaxf(t, -127.0f), 127.0f);
+            packed[e >> 2] |= ((uint32_t)((int)t & 0xFF)) << (8 * (e & 3));
+        }
+        q0 = packed[0];
+        q1 = packed[1];
+    }
+    if (csum) *csum = __dp4a((int)q0, 0x01010101, __dp4a((int)q1, 0x01010101, 0));
+}
+
 // ---------------------------------------------------------------------------
 // Per-token INT8 activation quantization ("Inference Quantization ch.1" §9.2;
 // "Kimi 2.7 MoE, 4-bit storage to INT8" §3.3):
@@ -43,44 +101,26 @@ __global__ void __launch_bounds__(kQuantThreads) quant_act_kernel(
     const uint4* xr = reinterpret_cast<const uint4*>(X + (size_t)m * ldx);
 
     uint4 raw[CPT];
-    float amax = 0.0f;
-    uint32_t bad = 0;
+    uint32_t am2 = 0;  // per-half maxima of the bf16 magnitudes
 #pragma unroll
     for (int i = 0; i < CPT; ++i) {
         const int c = i * kQuantThreads + tid;
         raw[i] = make_uint4(0, 0, 0, 0);
-        if (c < nchunk) {
-            raw[i] = __ldg(xr + c);
-            const uint32_t w[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
-#pragma unroll
-            for (int h = 0; h < 4; ++h) {
-                const uint32_t lo = w[h] & 0xFFFFu, hi = w[h] >> 16;
-                bad |= ((lo & 0x7F80u) == 0x7F80u) | ((hi & 0x7F80u) == 0x7F80u);
-                amax = fmaxf(amax, fabsf(bf16_bits_to_f32(lo)));
-                amax = fmaxf(amax, fabsf(bf16_bits_to_f32(hi)));
-            }
-        }
+        if (c < nchunk) raw[i] = __ldg(xr + c);
+        am2 = absmax_bf16x2(am2, raw[i].x);
+        am2 = absmax_bf16x2(am2, raw[i].y);
+        am2 = absmax_bf16x2(am2, raw[i].z);
+        am2 = absmax_bf16x2(am2, raw[i].w);
     }
-    // block-wide max / or
-    __shared__ float red_max[kQuantThreads / 32];
-    __shared__ uint32_t red_bad[kQuantThreads / 32];
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-        amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
-        bad |= __shfl_xor_sync(0xFFFFFFFFu, bad, off);
-    }
-    if ((tid & 31) == 0) {
-        red_max[tid >> 5] = amax;
-        red_bad[tid >> 5] = bad;
-    }
+    // block-wide maximum of the magnitude bits
+    __shared__ uint32_t red_max[kQuantThreads / 32];
+    uint32_t am = __reduce_max_sync(0xFFFFFFFFu, max(am2 & 0xFFFFu, am2 >> 16));
+    if ((tid & 31) == 0) red_max[tid >> 5] = am;
     __syncthreads();
-    amax = red_max[0];
-    bad = red_bad[0];
 #pragma unroll
-    for (int i = 1; i < kQuantThreads / 32; ++i) {
-        amax = fmaxf(amax, red_max[i]);
-        bad |= red_bad[i];
-    }
+    for (int i = 0; i < kQuantThreads / 32; ++i) am = max(am, red_max[i]);
+    const bool bad = am >= 0x7F80u;  // an Inf or NaN in the row
+    const float amax = bf16_bits_to_f32(am);
     const float s = __fdiv_rn(amax, 127.0f);
     const float d = (s > 0.0f) ? s : 1.0f;
     const float r_d = __frcp_rn(d);  // for the exact quotient rounding (rne_quotient)
@@ -90,18 +130,9 @@ __global__ void __launch_bounds__(kQuantThreads) quant_act_kernel(
     for (int i = 0; i < CPT; ++i) {
         const int c = i * kQuantThreads + tid;
         const bool live = c < nchunk;
-        const uint32_t w[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
-        uint32_t packed[2] = {0u, 0u};
+        uint32_t packed[2];
         int32_t csum = 0;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const uint32_t bits = (e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xFFFFu);
-            float t = rne_quotient(bf16_bits_to_f32(bits), d, r_d);
-            t = fminf(fmaxf(t, -127.0f), 127.0f);
-            const int qi = (int)t;
-            csum += qi;
-            packed[e >> 2] |= ((uint32_t)(qi & 0xFF)) << (8 * (e & 3));
-        }
+        quant_chunk8(raw[i], d, r_d, packed[0], packed[1], rowsum ? &csum : nullptr);
         if (live) {
             for (int j = 0; j < nrows_out; ++j) {
                 const int row = dest ? dest[(size_t)m * dest_k + j] : m;
@@ -146,38 +177,22 @@ __global__ void __launch_bounds__(kQuantThreads) quant_act_long_kernel(
     const int nchunk = K >> 3;
     const uint4* xr = reinterpret_cast<const uint4*>(X + (size_t)m * ldx);
 
-    float amax = 0.0f;
-    uint32_t bad = 0;
+    uint32_t am2 = 0;  // per-half maxima of the bf16 magnitudes
     for (int c = tid; c < nchunk; c += kQuantThreads) {
         const uint4 raw = __ldg(xr + c);
-        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-            const uint32_t lo = w[h] & 0xFFFFu, hi = w[h] >> 16;
-            bad |= ((lo & 0x7F80u) == 0x7F80u) | ((hi & 0x7F80u) == 0x7F80u);
-            amax = fmaxf(amax, fabsf(bf16_bits_to_f32(lo)));
-            amax = fmaxf(amax, fabsf(bf16_bits_to_f32(hi)));
-        }
+        am2 = absmax_bf16x2(am2, raw.x);
+        am2 = absmax_bf16x2(am2, raw.y);
+        am2 = absmax_bf16x2(am2, raw.z);
+        am2 = absmax_bf16x2(am2, raw.w);
     }
-    __shared__ float red_max[kQuantThreads / 32];
-    __shared__ uint32_t red_bad[kQuantThreads / 32];
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-        amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
-        bad |= __shfl_xor_sync(0xFFFFFFFFu, bad, off);
-    }
-    if ((tid & 31) == 0) {
-        red_max[tid >> 5] = amax;
-        red_bad[tid >> 5] = bad;
-    }
+    __shared__ uint32_t red_max[kQuantThreads / 32];
+    uint32_t am = __reduce_max_sync(0xFFFFFFFFu, max(am2 & 0xFFFFu, am2 >> 16));
+    if ((tid & 31) == 0) red_max[tid >> 5] = am;
     __syncthreads();
-    amax = red_max[0];
-    bad = red_bad[0];
 #pragma unroll
-    for (int i = 1; i < kQuantThreads / 32; ++i) {
-        amax = fmaxf(amax, red_max[i]);
-        bad |= red_bad[i];
-    }
+    for (int i = 0; i < kQuantThreads / 32; ++i) am = max(am, red_max[i]);
+    const bool bad = am >= 0x7F80u;  // an Inf or NaN in the row
+    const float amax = bf16_bits_to_f32(am);
     const float s = __fdiv_rn(amax, 127.0f);
     const float d = (s > 0.0f) ? s : 1.0f;
     const float r_d = __frcp_rn(d);  // for the exact quotient rounding (rne_quotient)
@@ -188,18 +203,9 @@ __global__ void __launch_bounds__(kQuantThreads) quant_act_long_kernel(
         const int c = c0 + tid;
         const bool live = c < nchunk;
         const uint4 raw = live ? __ldg(xr + c) : make_uint4(0, 0, 0, 0);
-        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-        uint32_t packed[2] = {0u, 0u};
+        uint32_t packed[2];
         int32_t csum = 0;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const uint32_t bits = (e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xFFFFu);
-            float t = rne_quotient(bf16_bits_to_f32(bits), d, r_d);
-            t = fminf(fmaxf(t, -127.0f), 127.0f);
-            const int qi = (int)t;
-            csum += qi;
-            packed[e >> 2] |= ((uint32_t)(qi & 0xFF)) << (8 * (e & 3));
-        }
+        quant_chunk8(raw, d, r_d, packed[0], packed[1], rowsum ? &csum : nullptr);
         if (live) *reinterpret_cast<uint2*>(q + (size_t)m * K + (size_t)c * 8) = make_uint2(packed[0], packed[1]);
         if (rowsum) {
             const int lanes = group >> 3;
@@ -233,8 +239,7 @@ __global__ void __launch_bounds__(32 * kQuantRowsPerCta) quant_act_rows_kernel(
     const uint4* xr = reinterpret_cast<const uint4*>(X + (size_t)m * ldx);
 
     uint4 raw[CPL];
-    float amax = 0.0f;
-    uint32_t bad = 0;
+    uint32_t am2 = 0;  // per-half maxima of the bf16 magnitudes
 #pragma unroll
     for (int i = 0; i < CPL; ++i) {
         const int c = i * 32 + lane;
@@ -243,20 +248,14 @@ __global__ void __launch_bounds__(32 * kQuantRowsPerCta) quant_act_rows_kernel(
     }
 #pragma unroll
     for (int i = 0; i < CPL; ++i) {
-        const uint32_t w[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-            const uint32_t lo = w[h] & 0xFFFFu, hi = w[h] >> 16;
-            bad |= ((lo & 0x7F80u) == 0x7F80u) | ((hi & 0x7F80u) == 0x7F80u);
-            amax = fmaxf(amax, fabsf(bf16_bits_to_f32(lo)));
-            amax = fmaxf(amax, fabsf(bf16_bits_to_f32(hi)));
-        }
+        am2 = absmax_bf16x2(am2, raw[i].x);
+        am2 = absmax_bf16x2(am2, raw[i].y);
+        am2 = absmax_bf16x2(am2, raw[i].z);
+        am2 = absmax_bf16x2(am2, raw[i].w);
     }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-        amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
-        bad |= __shfl_xor_sync(0xFFFFFFFFu, bad, off);
-    }
+    const uint32_t am = __reduce_max_sync(0xFFFFFFFFu, max(am2 & 0xFFFFu, am2 >> 16));
+    const bool bad = am >= 0x7F80u;  // an Inf or NaN in the row
+    const float amax = bf16_bits_to_f32(am);
     const float s = __fdiv_rn(amax, 127.0f);
     const float d = (s > 0.0f) ? s : 1.0f;
     const float r_d = __frcp_rn(d);  // for the exact quotient rounding (rne_quotient)
@@ -266,18 +265,9 @@ __global__ void __launch_bounds__(32 * kQuantRowsPerCta) quant_act_rows_kernel(
     for (int i = 0; i < CPL; ++i) {
         const int c = i * 32 + lane;
         const bool live = c < nchunk;
-        const uint32_t w[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
-        uint32_t packed[2] = {0u, 0u};
+        uint32_t packed[2];
         int32_t csum = 0;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const uint32_t bits = (e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xFFFFu);
-            float t = rne_quotient(bf16_bits_to_f32(bits), d, r_d);
-            t = fminf(fmaxf(t, -127.0f), 127.0f);
-            const int qi = (int)t;
-            csum += qi;
-            packed[e >> 2] |= ((uint32_t)(qi & 0xFF)) << (8 * (e & 3));
-        }
+        quant_chunk8(raw[i], d, r_d, packed[0], packed[1], rowsum ? &csum : nullptr);
         if (live) {
             for (int j = 0; j < nrows_out; ++j) {
                 const int row = dest ? dest[(size_t)m * dest_k + j] : m;
